@@ -1,0 +1,194 @@
+"""Seeded synthetic inputs for the deformable sampling-aggregation workloads.
+
+This module is shared by the CUDA path's tests and benchmark and by the CPU
+oracle's tests.  It draws random numbers (numpy PCG64, float64), applies the
+stated input recipe of each workload and rounds once to the workload dtype
+(torch `.to()`, round to nearest even).  It holds none of the operator's
+arithmetic: no bilinear read, no modulation softmax, no aggregation.
+
+The multi-scale recipe does contain the two module-side steps that produce the
+operator's inputs upstream of it: a 2-D reference point plus a pixel offset
+divided by the level size gives the normalised location, and the attention
+logits are normalised jointly over levels and points of a head.  They run here
+in numpy on the float64 draws, before rounding.
+
+Workload names state their sizes.  Shapes and distributions follow the
+DCNv4 note (Table 10 / Fig. 1 stage shapes), InternImage ch.5 (the 56/28/14/7
+stage hierarchy) and Deformable DETR (four feature levels, K points per level,
+M heads).  The features are synthetic stand-ins for backbone activations: no
+dataset or trained weights are used.
+"""
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+# integer codes of the C interface (dcn_dtype_t)
+DTYPE_CODES = {"f32": 0, "f16": 1, "bf16": 2}
+
+
+@dataclass(frozen=True)
+class DcnWorkload:
+    name: str
+    N: int
+    H: int
+    W: int
+    C: int
+    G: int
+    kh: int = 3
+    kw: int = 3
+    stride: int = 1
+    pad: int = 1
+    dil: int = 1
+    dtype: str = "f16"
+    offset_sigma: float = 2.0    # std of the pixel offsets
+    softmax_flag: int = 0        # 1: mask holds logits, softmax over K (DCNv3)
+
+    @property
+    def D(self):
+        return self.C // self.G
+
+    @property
+    def K(self):
+        return self.kh * self.kw
+
+    @property
+    def Ho(self):
+        return (self.H + 2 * self.pad - self.dil * (self.kh - 1) - 1) // self.stride + 1
+
+    @property
+    def Wo(self):
+        return (self.W + 2 * self.pad - self.dil * (self.kw - 1) - 1) // self.stride + 1
+
+    def taps(self):
+        """sampled taps: one per (output pixel, group, kernel point)."""
+        return self.N * self.Ho * self.Wo * self.G * self.K
+
+    def pixels(self):
+        return self.N * self.Ho * self.Wo
+
+    def compulsory_bytes(self):
+        """x, offsets, mask and out, each read or written once."""
+        es = DTYPES[self.dtype].itemsize
+        x = self.N * self.H * self.W * self.C
+        om = self.pixels() * self.G * self.K * 3
+        out = self.pixels() * self.C
+        return (x + om + out) * es
+
+
+@dataclass(frozen=True)
+class MsdaWorkload:
+    name: str
+    N: int
+    M: int
+    D: int
+    shapes: tuple             # ((H_l, W_l), ...)
+    K: int
+    Lq: int = 0               # 0: one query per pixel of all levels (encoder style)
+    dtype: str = "f32"
+    offset_sigma: float = 2.0  # std of the pixel offsets at each level
+
+    @property
+    def L(self):
+        return len(self.shapes)
+
+    @property
+    def S(self):
+        return sum(h * w for h, w in self.shapes)
+
+    @property
+    def queries(self):
+        return self.Lq if self.Lq else self.S
+
+    def taps(self):
+        return self.N * self.queries * self.M * self.L * self.K
+
+    def pixels(self):
+        return self.N * self.queries
+
+    def compulsory_bytes(self):
+        es = DTYPES[self.dtype].itemsize
+        value = self.N * self.S * self.M * self.D
+        loc = self.taps() * 2
+        w = self.taps()
+        out = self.N * self.queries * self.M * self.D
+        return (value + loc + w + out) * es
+
+
+WORKLOADS = {w.name: w for w in [
+    # DCNv3: softmax over the 9 taps, fp32
+    DcnWorkload("dcnv3_f32_1x14x14x64_g4", N=1, H=14, W=14, C=64, G=4, dtype="f32",
+                offset_sigma=1.0, softmax_flag=1),
+    # DCNv4 fp16 at the first-stage shape, batch 64 (the headline workload)
+    DcnWorkload("dcnv4_f16_64x56x56x64_g4", N=64, H=56, W=56, C=64, G=4, dtype="f16"),
+    # DCNv4 bf16 over the four stage shapes, G = C / 16
+    DcnWorkload("dcnv4_bf16_64x56x56x64_g4", N=64, H=56, W=56, C=64, G=4, dtype="bf16"),
+    DcnWorkload("dcnv4_bf16_64x28x28x128_g8", N=64, H=28, W=28, C=128, G=8, dtype="bf16"),
+    DcnWorkload("dcnv4_bf16_64x14x14x256_g16", N=64, H=14, W=14, C=256, G=16, dtype="bf16"),
+    DcnWorkload("dcnv4_bf16_64x7x7x512_g32", N=64, H=7, W=7, C=512, G=32, dtype="bf16"),
+    # DCNv4 fp16 at dense-prediction resolution with heavy-tailed offsets
+    DcnWorkload("dcnv4_f16_2x200x320x64_g4", N=2, H=200, W=320, C=64, G=4, dtype="f16",
+                offset_sigma=8.0),
+    # MSDeformAttn, four levels, encoder-style queries
+    MsdaWorkload("msda_f32_2x4lvl_m8_d32_k4", N=2, M=8, D=32,
+                 shapes=((100, 150), (50, 75), (25, 38), (13, 19)), K=4, dtype="f32"),
+]}
+
+HEADLINE = "dcnv4_f16_64x56x56x64_g4"
+
+
+def _round(a, dtype):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DTYPES[dtype])
+
+
+def dcn_inputs(w, seed=0):
+    """x [N,H,W,C] ~ U[-1,1]; offset [N,Ho,Wo,G,K,2] ~ N(0, sigma) px as (dx, dy);
+    mask [N,Ho,Wo,G,K] ~ N(0, 1) (unbounded m, or DCNv3 logits).  CPU tensors."""
+    rng = np.random.default_rng(seed)
+    x = rng.uniform(-1.0, 1.0, size=(w.N, w.H, w.W, w.C))
+    offset = rng.normal(0.0, w.offset_sigma, size=(w.N, w.Ho, w.Wo, w.G, w.K, 2))
+    mask = rng.normal(0.0, 1.0, size=(w.N, w.Ho, w.Wo, w.G, w.K))
+    return {"x": _round(x, w.dtype), "offset": _round(offset, w.dtype),
+            "mask": _round(mask, w.dtype)}
+
+
+def level_start_index(shapes):
+    """First value row of each level (levels concatenated row-major)."""
+    starts, s = [], 0
+    for h, wd in shapes:
+        starts.append(s)
+        s += h * wd
+    return starts
+
+
+def msda_inputs(w, seed=0):
+    """value [N,S,M,D] ~ U[-1,1]; one reference point per (n, q) ~ U[0,1]^2 shared
+    by heads, levels and points; pixel offsets ~ N(0, sigma) per (m, l, k) divided
+    by (W_l, H_l); logits ~ N(0,1) normalised jointly over (l, k) per head."""
+    rng = np.random.default_rng(seed)
+    Lq = w.queries
+    value = rng.uniform(-1.0, 1.0, size=(w.N, w.S, w.M, w.D))
+    ref = rng.uniform(0.0, 1.0, size=(w.N, Lq, 2))
+    dp = rng.normal(0.0, w.offset_sigma, size=(w.N, Lq, w.M, w.L, w.K, 2))
+    logits = rng.normal(0.0, 1.0, size=(w.N, Lq, w.M, w.L, w.K))
+    size_wh = np.array([[wd, h] for h, wd in w.shapes], dtype=np.float64)  # [L, 2]
+    loc = ref[:, :, None, None, None, :] + dp / size_wh[None, None, None, :, None, :]
+    flat = logits.reshape(w.N, Lq, w.M, w.L * w.K)
+    e = np.exp(flat - flat.max(axis=-1, keepdims=True))
+    attn = (e / e.sum(axis=-1, keepdims=True)).reshape(logits.shape)
+    return {
+        "value": _round(value, w.dtype),
+        "spatial_shapes": torch.tensor(w.shapes, dtype=torch.int64),
+        "level_start": torch.tensor(level_start_index(w.shapes), dtype=torch.int64),
+        "loc": _round(loc, w.dtype),
+        "attn": _round(attn, w.dtype),
+        "logits": logits,
+    }
+
+
+def scaled(w, **changes):
+    """A copy of workload `w` with some fields replaced (e.g. a smaller batch)."""
+    fields = dict(w.__dict__)
+    fields.update(changes)
+    return type(w)(**fields)

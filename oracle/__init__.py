@@ -1,0 +1,111 @@
+"""CPU oracle for the deformable sampling-aggregation path.
+
+TEST INFRASTRUCTURE.  This package is the plain, slow, float64 definition the
+CUDA library is checked against.  Only the test suite, the smoke check and the
+benchmark's CPU-baseline leg may import it; the product path never does, and
+it imports nothing from the product package.
+
+`dcn_forward_ref` and `msda_forward_ref` call the C loop nests in
+dcn_oracle.c through ctypes.  Inputs may be numpy arrays or torch CPU tensors
+in any floating dtype; each value is converted exactly to float64 before the
+arithmetic (every fp16, bf16 and fp32 value is representable in float64).
+
+Parity status: every function here is pinned by the CPU tests against worked
+examples printed on the pages, closed forms, invariants and library routines
+(torch grid_sample / conv2d in float64); no function is parity-unpinned.
+"""
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+from . import scalar  # noqa: F401  (re-exported for the tests)
+
+_lib = None
+
+
+def bind(lib):
+    """Declare the C signatures on a loaded oracle library and return it."""
+    dp = ctypes.POINTER(ctypes.c_double)
+    lp = ctypes.POINTER(ctypes.c_longlong)
+    L = ctypes.c_long
+    lib.oracle_dcn_forward.argtypes = [dp, dp, dp, dp] + [L] * 10 + [ctypes.c_int]
+    lib.oracle_dcn_forward.restype = ctypes.c_int
+    lib.oracle_msda_forward.argtypes = [dp, lp, lp, dp, dp, dp] + [L] * 7
+    lib.oracle_msda_forward.restype = ctypes.c_int
+    lib.oracle_out_size.argtypes = [L] * 5
+    lib.oracle_out_size.restype = L
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = bind(ctypes.CDLL(_build.build()))
+    return _lib
+
+
+def _as_f64(a):
+    """Exact float64 copy of a numpy array or torch tensor (any float dtype)."""
+    if hasattr(a, "detach"):            # torch tensor (bf16 has no numpy dtype)
+        import torch
+        a = a.detach().to("cpu", torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a, ctype=ctypes.c_double):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def out_size(n_in, k, stride, pad, dil):
+    return int(_load().oracle_out_size(n_in, k, stride, pad, dil))
+
+
+def dcn_forward_ref(x, offset, mask, kh, kw, stride=1, pad=1, dil=1, softmax_flag=0,
+                    groups=None):
+    """float64 DCNv3/DCNv4 forward.
+
+    x [N, H, W, C], offset [N, Ho, Wo, G, K, 2], mask [N, Ho, Wo, G, K]
+    -> out [N, Ho, Wo, C] float64.  G is taken from mask.shape[3] unless given.
+    """
+    x = _as_f64(x)
+    offset = _as_f64(offset)
+    mask = _as_f64(mask)
+    N, H, W, C = x.shape
+    G = groups if groups is not None else mask.shape[3]
+    Ho = out_size(H, kh, stride, pad, dil)
+    Wo = out_size(W, kw, stride, pad, dil)
+    K = kh * kw
+    assert offset.size == N * Ho * Wo * G * K * 2, "offset has the wrong size"
+    assert mask.size == N * Ho * Wo * G * K, "mask has the wrong size"
+    out = np.zeros((N, Ho, Wo, C), dtype=np.float64)
+    rc = _load().oracle_dcn_forward(_ptr(x), _ptr(offset), _ptr(mask), _ptr(out),
+                                    N, H, W, C, G, kh, kw, stride, pad, dil,
+                                    int(softmax_flag))
+    if rc != 0:
+        raise ValueError("oracle_dcn_forward rejected its arguments")
+    return out
+
+
+def msda_forward_ref(value, spatial_shapes, level_start, loc, attn):
+    """float64 MSDeformAttn core forward.
+
+    value [N, S, M, D], spatial_shapes [L, 2] as (H, W), level_start [L],
+    loc [N, Lq, M, L, K, 2] as (u, v), attn [N, Lq, M, L, K]
+    -> out [N, Lq, M * D] float64.
+    """
+    value = _as_f64(value)
+    loc = _as_f64(loc)
+    attn = _as_f64(attn)
+    shapes = np.ascontiguousarray(np.asarray(spatial_shapes, dtype=np.int64))
+    starts = np.ascontiguousarray(np.asarray(level_start, dtype=np.int64))
+    N, S, M, D = value.shape
+    _, Lq, _, L, K = attn.shape
+    assert loc.shape == (N, Lq, M, L, K, 2), "loc has the wrong shape"
+    out = np.zeros((N, Lq, M * D), dtype=np.float64)
+    rc = _load().oracle_msda_forward(_ptr(value), _ptr(shapes, ctypes.c_longlong),
+                                     _ptr(starts, ctypes.c_longlong), _ptr(loc),
+                                     _ptr(attn), _ptr(out), N, S, Lq, M, D, L, K)
+    if rc != 0:
+        raise ValueError("oracle_msda_forward rejected its arguments")
+    return out
