@@ -1,0 +1,513 @@
+"""Benchmark of the deformable sampling-aggregation forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--workload NAME]
+
+One step is one dcn_forward (or msda_forward) call over one full batch of the
+workload; the default workload is DCNv4 fp16, N=64, 56x56, C=64, G=4, 3x3.
+Prints ONE JSON line on stdout (rank 0); diagnostics go to stderr.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
+and a device synchronisation on both sides, timed with CUDA events on the
+launch stream.  The steps rotate over enough independent input/output sets
+that their total exceeds three L2 caches, so every step reads from HBM.
+Multi-GPU (torchrun): each rank runs its own batch (weak scaling, no data
+collective); the time is the maximum over ranks and `value` counts the taps
+of all ranks.
+
+`--impl reference` times the float64 CPU oracle (the reference arm) on rank 0
+over a bounded sample of the same workload per step.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gen  # noqa: E402
+
+METRIC = ("sampled taps/s & achieved HBM GB/s vs peak "
+          "(DCNv4 fp16 fwd, 64×56²×64, G=4)")
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic of the timed kernel from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum per launch, headline workload), with the hash of the
+# kernel sources it was taken on; reported as null once the sources change.
+NCU_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None}
+
+KERNEL_SOURCES = [
+    "deformable_attention_sampling_b200/csrc/common.cuh",
+    "deformable_attention_sampling_b200/csrc/dcn_fwd.cuh",
+    "deformable_attention_sampling_b200/csrc/msda_fwd.cuh",
+    "deformable_attention_sampling_b200/csrc/dcn_abi.cu",
+    "include/dcn.h",
+]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock, max clock and clock-event reasons with NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            props = torch.cuda.get_device_properties(device_index)
+            handle = None
+            for lookup in (
+                    lambda: pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid)),
+                    lambda: pynvml.nvmlDeviceGetHandleByPciBusId(
+                        f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:"
+                        f"{props.pci_device_id:02X}.0"),
+                    lambda: pynvml.nvmlDeviceGetHandleByIndex(device_index)):
+                try:
+                    handle = lookup()
+                    break
+                except Exception:
+                    continue
+            if handle is None:
+                raise RuntimeError("no NVML handle for the CUDA device")
+            self.handle = handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:   # no NVML: report the clocks as unavailable
+            self.nvml = None
+            self.error = str(e)
+
+    def _sample(self):
+        n = self.nvml
+        sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+        try:
+            reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+        except AttributeError:
+            reasons = n.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+        self.samples.append((sm, reasons))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception as e:
+                self.error = str(e)
+                return
+            time.sleep(0.002)
+
+    def start(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+            try:
+                self._sample()      # at least one sample right at the end
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "error": self.error}
+        mask = 0
+        for _, r in self.samples:
+            mask |= int(r)
+        reasons = [name for bit, name in self.REASONS.items() if mask & bit]
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ runners
+
+class DcnRunner:
+    def __init__(self, w, seed, device):
+        import deformable_attention_sampling_b200 as dcnb
+        self.dcnb = dcnb
+        self.w = w
+        self.host = gen.dcn_inputs(w, seed=seed)
+        self.device = device
+        self.code = gen.DTYPE_CODES[w.dtype]
+        self.lib = dcnb.library()
+
+    def alloc_set(self):
+        d = {k: v.to(self.device) for k, v in self.host.items()}
+        d["out"] = torch.empty((self.w.N, self.w.Ho, self.w.Wo, self.w.C),
+                               dtype=self.host["x"].dtype, device=self.device)
+        return d
+
+    def launcher(self, s, stream):
+        """A closure issuing one step on set s with pre-resolved arguments."""
+        w, lib = self.w, self.lib
+        args = (s["x"].data_ptr(), s["offset"].data_ptr(), s["mask"].data_ptr(),
+                s["out"].data_ptr(), w.N, w.H, w.W, w.C, w.G, w.kh, w.kw, w.stride, w.pad,
+                w.dil, w.softmax_flag, self.code, stream)
+
+        def go():
+            st = lib.dcn_forward(*args)
+            if st != 0:
+                raise self.dcnb.DcnError(st, "dcn_forward")
+        return go
+
+    def inputs_of(self, s):
+        return [(s["x"], self.host["x"]), (s["offset"], self.host["offset"]),
+                (s["mask"], self.host["mask"])]
+
+
+class MsdaRunner:
+    def __init__(self, w, seed, device):
+        import deformable_attention_sampling_b200 as dcnb
+        self.dcnb = dcnb
+        self.w = w
+        self.host = {k: v for k, v in gen.msda_inputs(w, seed=seed).items() if k != "logits"}
+        self.device = device
+        self.code = gen.DTYPE_CODES[w.dtype]
+        self.lib = dcnb.library()
+
+    def alloc_set(self):
+        d = {k: v.to(self.device) for k, v in self.host.items()}
+        d["out"] = torch.empty((self.w.N, self.w.queries, self.w.M * self.w.D),
+                               dtype=self.host["value"].dtype, device=self.device)
+        return d
+
+    def launcher(self, s, stream):
+        w, lib = self.w, self.lib
+        args = (s["value"].data_ptr(), s["spatial_shapes"].data_ptr(),
+                s["level_start"].data_ptr(), s["loc"].data_ptr(), s["attn"].data_ptr(),
+                s["out"].data_ptr(), w.N, w.queries, w.M, w.D, w.L, w.K, self.code, stream)
+
+        def go():
+            st = lib.msda_forward(*args)
+            if st != 0:
+                raise self.dcnb.DcnError(st, "msda_forward")
+        return go
+
+    def inputs_of(self, s):
+        return [(s[k], self.host[k]) for k in ("value", "spatial_shapes", "level_start", "loc",
+                                               "attn")]
+
+
+def make_runner(w, seed, device):
+    return (DcnRunner if isinstance(w, gen.DcnWorkload) else MsdaRunner)(w, seed, device)
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_step(w, seed):
+    """Run the float64 oracle once on workload w; returns (seconds, taps)."""
+    import oracle
+    if isinstance(w, gen.DcnWorkload):
+        inp = gen.dcn_inputs(w, seed=seed)
+        t = time.perf_counter()
+        oracle.dcn_forward_ref(inp["x"], inp["offset"], inp["mask"], w.kh, w.kw, w.stride,
+                               w.pad, w.dil, w.softmax_flag)
+    else:
+        inp = gen.msda_inputs(w, seed=seed)
+        t = time.perf_counter()
+        oracle.msda_forward_ref(inp["value"], inp["spatial_shapes"], inp["level_start"],
+                                inp["loc"], inp["attn"])
+    return time.perf_counter() - t, w.taps()
+
+
+def sample_of(w, n_images):
+    """A bounded sample of workload w with the same per-tap work: fewer batch
+    items (DCN) or fewer queries (MSDA)."""
+    if isinstance(w, gen.DcnWorkload):
+        return gen.scaled(w, N=max(1, min(w.N, n_images)))
+    return gen.scaled(w, N=1, Lq=max(1, min(w.queries, n_images * 64)))
+
+
+def cpu_baseline(w, budget_s=10.0):
+    """The oracle as it stands, single-threaded, on a bounded sample of the
+    workload, repeated until about `budget_s` seconds of CPU work."""
+    s = sample_of(w, 8)
+    total_t, total_taps, reps = 0.0, 0, 0
+    while total_t < budget_s or reps == 0:
+        dt, taps = oracle_step(s, seed=reps)
+        total_t += dt
+        total_taps += taps
+        reps += 1
+    desc = (f"{reps} x oracle on {s.name} with N={s.N}" +
+            (f", Lq={s.queries}" if isinstance(s, gen.MsdaWorkload) else "") +
+            f" ({s.taps()} taps each), single thread, float64")
+    return {"value": total_taps / total_t, "unit": "taps/s", "cores": 1, "kind": "oracle",
+            "sample": desc, "host_cpus": os.cpu_count()}
+
+
+# ------------------------------------------------------------------ main arms
+
+def setup_distributed():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(f"cuda:{local}"))
+    return world, rank, local
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world, device):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[device.index])
+    torch.cuda.synchronize(device)
+
+
+def run_b200(args):
+    world, rank, local = setup_distributed()
+    device = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(device)
+    w = gen.WORKLOADS[args.workload]
+    import deformable_attention_sampling_b200 as dcnb
+    from deformable_attention_sampling_b200 import build as dcn_build
+    if not os.path.exists(dcn_build.LIB):
+        raise RuntimeError("libdcn_b200.so is not built (python -m "
+                           "deformable_attention_sampling_b200.build)")
+
+    runner = make_runner(w, seed=1000 + rank, device=device)
+    bytes_per_step = w.compulsory_bytes()
+    n_sets = max(2, int(np.ceil(3 * L2_BYTES / bytes_per_step)))
+    sets = [runner.alloc_set() for _ in range(n_sets)]
+    stream = torch.cuda.current_stream(device)
+    handle = int(stream.cuda_stream)
+    launch = [runner.launcher(s, handle) for s in sets]
+    log(f"[rank {rank}] workload {w.name}: {w.taps()} taps, {bytes_per_step / 1e6:.2f} MB "
+        f"compulsory per step, {n_sets} rotating sets")
+
+    for i in range(args.warmup):
+        launch[i % n_sets]()
+    barrier(world, device)
+
+    sampler = ClockSampler(local)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    launches_before = dcnb.dcn_launch_count()
+    sampler.start()
+    start.record(stream)
+    for i in range(args.steps):
+        launch[i % n_sets]()
+    end.record(stream)
+    end.synchronize()
+    sampler.stop()
+    launches = dcnb.dcn_launch_count() - launches_before
+    barrier(world, device)
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(ms_local, world, device)
+    ms_per_step = ms / args.steps
+
+    # end to end through the public call with host buffers: H2D of the step's
+    # inputs from pinned memory, the call, D2H of the output, every step
+    e2e_steps = min(args.steps, 200)
+    pinned_out = torch.empty(sets[0]["out"].shape, dtype=sets[0]["out"].dtype).pin_memory()
+    pinned_in = [(dev, host.pin_memory()) for dev, host in runner.inputs_of(sets[0])]
+    h2d = sum(h.numel() * h.element_size() for _, h in pinned_in)
+    d2h = pinned_out.numel() * pinned_out.element_size()
+    for _ in range(2):
+        for dev, host in pinned_in:
+            dev.copy_(host, non_blocking=True)
+        launch[0]()
+        pinned_out.copy_(sets[0]["out"], non_blocking=True)
+    barrier(world, device)
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(e2e_steps):
+        for dev, host in pinned_in:
+            dev.copy_(host, non_blocking=True)
+        launch[0]()
+        pinned_out.copy_(sets[0]["out"], non_blocking=True)
+    e_end.record(stream)
+    e_end.synchronize()
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world, device) / e2e_steps
+    barrier(world, device)
+
+    taps_total = w.taps() * world
+    value = taps_total / (ms_per_step * 1e-3)
+    peak, peak_src = measured_hbm_peak()
+    achieved = bytes_per_step / (ms_local / args.steps * 1e-3) / 1e9
+    traffic = None
+    if (NCU_TRAFFIC["source_sha256"] == kernel_source_hash()
+            and w.name == gen.HEADLINE):
+        traffic = NCU_TRAFFIC["bytes_per_launch"]
+
+    result = None
+    if rank == 0:
+        kernel = "dcn_fwd_kernel" if isinstance(w, gen.DcnWorkload) else "msda_fwd_kernel"
+        config = {"workload": w.name, "global_batch": w.N * world,
+                  "per_gpu_batch": w.N, "dtype_storage": w.dtype, "accumulate": "f32",
+                  "l2": f"{n_sets} rotating input/output sets ({n_sets * bytes_per_step / 1e6:.0f} MB"
+                        f" > L2 {L2_BYTES / 1e6:.0f} MB)",
+                  "parallelism": f"dp{world}" if world > 1 else "single GPU"}
+        if isinstance(w, gen.DcnWorkload):
+            config.update({"H": w.H, "W": w.W, "C": w.C, "G": w.G, "kernel": f"{w.kh}x{w.kw}",
+                           "stride": w.stride, "pad": w.pad, "dil": w.dil,
+                           "softmax": bool(w.softmax_flag), "offset_sigma_px": w.offset_sigma})
+        else:
+            config.update({"M": w.M, "D": w.D, "levels": [list(s) for s in w.shapes],
+                           "K": w.K, "Lq": w.queries})
+        result = {
+            "metric": METRIC if w.name == gen.HEADLINE else f"sampled taps/s ({w.name})",
+            "value": value,
+            "unit": "taps/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": w.dtype,
+            "data": "synthetic (seeded generator; no dataset or weights)",
+            "config": config,
+            "pixels_per_s": w.pixels() * world / (ms_per_step * 1e-3),
+            "hbm_gbs": achieved,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": kernel, "algorithmic_bytes_per_launch": bytes_per_step,
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_src == "measured" else "fallback 6.65 TB/s"},
+            "e2e": {"value": taps_total / (e2e_ms * 1e-3), "unit": "taps/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms, "steps": e2e_steps},
+            "gpu_launches": int(launches),
+            "clocks": sampler.summary(),
+        }
+        if world == 1:
+            result["cpu_baseline"] = cpu_baseline(w)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[device.index])
+        dist.destroy_process_group()
+    return result
+
+
+def run_reference(args):
+    """The reference arm: the float64 CPU oracle, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return None
+    w = gen.WORKLOADS[args.workload]
+    # size one step so that warm-up plus timed steps take about a minute
+    probe = sample_of(w, 1)
+    dt, taps = oracle_step(probe, seed=0)
+    rate = taps / dt
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    if isinstance(w, gen.DcnWorkload):
+        per_image = w.taps() / w.N
+        n = max(1, min(w.N, int(budget * rate / per_image)))
+        if budget * rate < per_image:     # less than one image: crop its rows
+            rows = max(1, int(w.H * budget * rate / per_image))
+            step_w = gen.scaled(w, N=1, H=rows)
+        else:
+            step_w = gen.scaled(w, N=n)
+    else:
+        per_query = w.taps() / (w.N * w.queries)
+        q = max(1, min(w.queries, int(budget * rate / per_query)))
+        step_w = gen.scaled(w, N=1, Lq=q)
+    for i in range(args.warmup):
+        oracle_step(step_w, seed=i)
+    total_t, total_taps = 0.0, 0
+    for i in range(args.steps):
+        t, taps = oracle_step(step_w, seed=args.warmup + i)
+        total_t += t
+        total_taps += taps
+    value = total_taps / total_t
+    sample = (f"each step: oracle on {step_w.name} with N={step_w.N}"
+              + (f", H={step_w.H}" if isinstance(step_w, gen.DcnWorkload) else
+                 f", Lq={step_w.queries}")
+              + f" ({step_w.taps()} taps), single thread, float64")
+    return {
+        "impl": "reference",
+        "metric": METRIC if w.name == gen.HEADLINE else f"sampled taps/s ({w.name})",
+        "value": value,
+        "unit": "taps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_t / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded generator; no dataset or weights)",
+        "config": {"workload": w.name, "global_batch": w.N, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "taps/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "taps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20000)
+    p.add_argument("--warmup", type=int, default=200)
+    p.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    p.add_argument("--workload", default=gen.HEADLINE, choices=sorted(gen.WORKLOADS))
+    args = p.parse_args()
+    if args.warmup < 3:
+        p.error("--warmup must be at least 3")
+    result = run_reference(args) if args.impl == "reference" else run_b200(args)
+    if result is not None:
+        print(json.dumps(result), flush=True)
+
+
+if __name__ == "__main__":
+    main()

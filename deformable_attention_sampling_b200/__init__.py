@@ -1,0 +1,33 @@
+"""Deformable sampling-aggregation on NVIDIA B200 (sm_100a).
+
+DCNv3 / DCNv4 deformable convolution core and the multi-scale deformable
+attention (MSDeformAttn) core, forward, as hand-written CUDA kernels behind a
+C interface (include/dcn.h, libdcn_b200.so).  This package is the thin Python
+binding: it marshals pointers, sizes and streams and runs nothing itself.
+
+    import deformable_attention_sampling_b200 as dcnb
+    out = dcnb.dcn(x, offset, mask)          # torch CUDA tensors, NHWC
+    out = dcnb.msda(value, shapes, starts, loc, attn)
+"""
+from ._binding import (  # noqa: F401
+    DCN_ERR_CUDA,
+    DCN_ERR_INVALID_ARG,
+    DCN_ERR_MISALIGNED,
+    DCN_ERR_UNSUPPORTED,
+    DCN_OK,
+    DTYPE_CODES,
+    LIB_PATH,
+    SIGNATURES,
+    DcnError,
+    dcn,
+    dcn_forward,
+    dcn_last_cuda_error,
+    dcn_launch_count,
+    dcn_output_size,
+    dcn_status_string,
+    dcn_version,
+    dtype_code,
+    library,
+    msda,
+    msda_forward,
+)

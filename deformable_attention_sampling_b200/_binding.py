@@ -1,0 +1,205 @@
+"""ctypes binding of libdcn_b200.so (include/dcn.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C interface.  Pointer arguments may be integers (device
+addresses) or objects with a ``data_ptr()`` method (torch tensors); stream
+arguments may be None (torch's current stream), an integer handle, or an object
+with a ``cuda_stream`` attribute.  A non-OK status raises DcnError.
+
+There is no fallback: when the shared library is missing the first call
+raises RuntimeError naming the build command.
+"""
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "_lib", "libdcn_b200.so")
+
+DCN_OK = 0
+DCN_ERR_INVALID_ARG = -1
+DCN_ERR_UNSUPPORTED = -2
+DCN_ERR_MISALIGNED = -3
+DCN_ERR_CUDA = -4
+DTYPE_CODES = {"f32": 0, "f16": 1, "bf16": 2}
+
+# every symbol include/dcn.h declares, with its ctypes signature
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+SIGNATURES = {
+    "dcn_forward": (_I, [_VP, _VP, _VP, _VP] + [_I] * 12 + [_VP]),
+    "msda_forward": (_I, [_VP] * 6 + [_I] * 7 + [_VP]),
+    "dcn_output_size": (_I, [_I] * 5),
+    "dcn_status_string": (ctypes.c_char_p, [_I]),
+    "dcn_last_cuda_error": (_I, []),
+    "dcn_launch_count": (ctypes.c_uint64, []),
+    "dcn_version": (_I, []),
+}
+
+_lib = None
+
+
+class DcnError(RuntimeError):
+    """A dcn_status_t other than DCN_OK."""
+
+    def __init__(self, status, where):
+        self.status = status
+        text = _load().dcn_status_string(status).decode()
+        detail = ""
+        if status == DCN_ERR_CUDA:
+            detail = f" (cudaError {_load().dcn_last_cuda_error()})"
+        super().__init__(f"{where}: {text}{detail} [status {status}]")
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m deformable_attention_sampling_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def library():
+    """The loaded ctypes library (loads it on first use)."""
+    return _load()
+
+
+def _ptr(p):
+    if p is None:
+        return None
+    if isinstance(p, int):
+        return p
+    return int(p.data_ptr())
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(s, int):
+        return s
+    return int(s.cuda_stream)
+
+
+def _check(status, where):
+    if status != DCN_OK:
+        raise DcnError(status, where)
+
+
+def dcn_forward(x, offset, mask, out, N, H, W, C, G, kh, kw, stride, pad, dil,
+                softmax_flag, dtype, stream=None):
+    """C dcn_forward; raises DcnError on a non-OK status."""
+    _check(_load().dcn_forward(_ptr(x), _ptr(offset), _ptr(mask), _ptr(out), N, H, W, C, G,
+                               kh, kw, stride, pad, dil, softmax_flag, dtype, _stream(stream)),
+           "dcn_forward")
+
+
+def msda_forward(value, spatial_shapes, level_start, sampling_loc, attn_w, out, N, Lq, M, D,
+                 L, K, dtype, stream=None):
+    """C msda_forward; raises DcnError on a non-OK status."""
+    _check(_load().msda_forward(_ptr(value), _ptr(spatial_shapes), _ptr(level_start),
+                                _ptr(sampling_loc), _ptr(attn_w), _ptr(out), N, Lq, M, D, L,
+                                K, dtype, _stream(stream)),
+           "msda_forward")
+
+
+def dcn_output_size(n_in, k, stride, pad, dil):
+    return int(_load().dcn_output_size(n_in, k, stride, pad, dil))
+
+
+def dcn_status_string(status):
+    return _load().dcn_status_string(status).decode()
+
+
+def dcn_last_cuda_error():
+    return int(_load().dcn_last_cuda_error())
+
+
+def dcn_launch_count():
+    return int(_load().dcn_launch_count())
+
+
+def dcn_version():
+    return int(_load().dcn_version())
+
+
+# ------------------------------------------------------------ tensor helpers
+
+def dtype_code(t):
+    """dcn_dtype_t of a torch tensor."""
+    import torch
+    codes = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+    if t.dtype not in codes:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def _require(cond, msg):
+    if not cond:
+        raise ValueError(msg)
+
+
+def dcn(x, offset, mask, kh=3, kw=3, stride=1, pad=1, dil=1, softmax_flag=0, out=None,
+        stream=None):
+    """dcn_forward on torch CUDA tensors; allocates `out` when not given.
+
+    x [N, H, W, C], offset [N, Ho, Wo, G, K, 2], mask [N, Ho, Wo, G, K], all of
+    one dtype (float32 / float16 / bfloat16), contiguous, on one CUDA device.
+    """
+    import torch
+    _require(x.dim() == 4 and mask.dim() == 5 and offset.dim() == 6,
+             "expected x [N,H,W,C], offset [N,Ho,Wo,G,K,2], mask [N,Ho,Wo,G,K]")
+    N, H, W, C = x.shape
+    G = mask.shape[3]
+    Ho = dcn_output_size(H, kh, stride, pad, dil)
+    Wo = dcn_output_size(W, kw, stride, pad, dil)
+    K = kh * kw
+    _require(tuple(offset.shape) == (N, Ho, Wo, G, K, 2), "offset has the wrong shape")
+    _require(tuple(mask.shape) == (N, Ho, Wo, G, K), "mask has the wrong shape")
+    _require(offset.dtype == x.dtype and mask.dtype == x.dtype, "mixed dtypes")
+    _require(x.is_cuda and offset.is_cuda and mask.is_cuda, "tensors must be on a CUDA device")
+    _require(x.is_contiguous() and offset.is_contiguous() and mask.is_contiguous(),
+             "tensors must be contiguous")
+    if out is None:
+        out = torch.empty((N, Ho, Wo, C), dtype=x.dtype, device=x.device)
+    _require(tuple(out.shape) == (N, Ho, Wo, C) and out.dtype == x.dtype and out.is_contiguous(),
+             "out has the wrong shape, dtype or layout")
+    dcn_forward(x, offset, mask, out, N, H, W, C, G, kh, kw, stride, pad, dil, softmax_flag,
+                dtype_code(x), stream)
+    return out
+
+
+def msda(value, spatial_shapes, level_start, sampling_loc, attn_w, out=None, stream=None):
+    """msda_forward on torch CUDA tensors; allocates `out` when not given.
+
+    value [N, S, M, D], spatial_shapes [L, 2] int64 (H, W), level_start [L] int64,
+    sampling_loc [N, Lq, M, L, K, 2], attn_w [N, Lq, M, L, K].
+    """
+    import torch
+    _require(value.dim() == 4 and attn_w.dim() == 5 and sampling_loc.dim() == 6,
+             "expected value [N,S,M,D], loc [N,Lq,M,L,K,2], attn [N,Lq,M,L,K]")
+    N, S, M, D = value.shape
+    _, Lq, _, L, K = attn_w.shape
+    _require(tuple(sampling_loc.shape) == (N, Lq, M, L, K, 2), "sampling_loc has the wrong shape")
+    _require(tuple(attn_w.shape[:3]) == (N, Lq, M), "attn_w has the wrong shape")
+    _require(tuple(spatial_shapes.shape) == (L, 2) and tuple(level_start.shape) == (L,),
+             "spatial_shapes / level_start have the wrong shape")
+    _require(spatial_shapes.dtype == torch.int64 and level_start.dtype == torch.int64,
+             "spatial_shapes / level_start must be int64")
+    _require(sampling_loc.dtype == value.dtype and attn_w.dtype == value.dtype, "mixed dtypes")
+    for t in (value, spatial_shapes, level_start, sampling_loc, attn_w):
+        _require(t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty((N, Lq, M * D), dtype=value.dtype, device=value.device)
+    _require(tuple(out.shape) == (N, Lq, M * D) and out.dtype == value.dtype and out.is_contiguous(),
+             "out has the wrong shape, dtype or layout")
+    msda_forward(value, spatial_shapes, level_start, sampling_loc, attn_w, out, N, Lq, M, D, L,
+                 K, dtype_code(value), stream)
+    return out

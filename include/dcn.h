@@ -1,0 +1,150 @@
+/*
+ * dcn.h - C interface of libdcn_b200.so: deformable sampling-aggregation
+ * (DCNv3 / DCNv4 core) and multi-scale deformable attention (MSDeformAttn core)
+ * forward on NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates nothing, never synchronises, and launches its kernels
+ *     asynchronously on `stream` (a cudaStream_t; NULL is the legacy default
+ *     stream).  The caller keeps the buffers alive until the stream has run.
+ *   - Tensors are contiguous, row-major, in the layouts stated per call.
+ *   - `dtype` (dcn_dtype_t) applies to every floating tensor of the call
+ *     (inputs and output).  Arithmetic is float32 throughout: 16-bit inputs are
+ *     widened exactly, products and sums are float32, and the output is rounded
+ *     once, to nearest even.
+ *   - `out` must not overlap any input (DCN_ERR_INVALID_ARG).
+ *   - No C++ exception crosses this interface; every entry point returns a
+ *     dcn_status_t.  On an error nothing is launched and `out` is untouched,
+ *     except DCN_ERR_CUDA, which reports a failed launch.
+ *   - Thread safety: calls are independent and may come from several host
+ *     threads; each runs on the stream it is given.
+ */
+#ifndef DCN_B200_H
+#define DCN_B200_H
+
+#include <stdint.h>
+
+/* symbols of the shared library (it is built with hidden default visibility) */
+#if defined(__GNUC__)
+#define DCN_API __attribute__((visibility("default")))
+#else
+#define DCN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { DCN_F32 = 0, DCN_F16 = 1, DCN_BF16 = 2 } dcn_dtype_t;
+
+typedef enum {
+    DCN_OK = 0,
+    DCN_ERR_INVALID_ARG = -1,  /* bad dimension, null pointer, unknown dtype, aliasing */
+    DCN_ERR_UNSUPPORTED = -2,  /* valid request beyond the library's stated limits */
+    DCN_ERR_MISALIGNED = -3,   /* a pointer not aligned to its element size */
+    DCN_ERR_CUDA = -4          /* the kernel launch failed (see dcn_last_cuda_error) */
+} dcn_status_t;
+
+/*
+ * dcn_forward - DCNv3 / DCNv4 deformable sampling-aggregation, forward.
+ *
+ * Defined by "InternImage: Deformable Convolutions at Scale" ch.1-4 (learned
+ * offsets, bilinear read with zero padding, groups) and the "DCNv4" note,
+ * "Why Is Sampling Just 9 Points Still Slow?" (y_g(p0) = sum_k m_gk x_g(p0 +
+ * p_k + dp_gk)) and "1. Remove Softmax".  For every output pixel (oy, ox),
+ * group g < G and channel c < D = C / G:
+ *
+ *   out[n][oy][ox][g*D + c] = sum_{ix < kw, iy < kh} m[k] * B(x[n][.][.][g*D + c], px, py)
+ *     k  = ix * kh + iy
+ *     px = ox*stride - pad + ix*dil + offset[n][oy][ox][g][k][0]
+ *     py = oy*stride - pad + iy*dil + offset[n][oy][ox][g][k][1]
+ *     m[k] = mask[n][oy][ox][g][k]                       (softmax_flag = 0, DCNv4)
+ *     m[k] = softmax over k of mask[n][oy][ox][g][.]     (softmax_flag = 1, DCNv3)
+ *   B(f, px, py): bilinear read, corners floor(p) and floor(p) + 1 with weights
+ *   (1-a)(1-b), a(1-b), (1-a)b, ab (a, b the fractional parts); corners outside
+ *   the map read 0 (no clamping, no renormalisation).
+ *
+ * Layouts (channels-last):
+ *   x      [N][H][W][C]
+ *   offset [N][Ho][Wo][G][K][2]   (dx, dy) in pixels, x along W, K = kh * kw
+ *   mask   [N][Ho][Wo][G][K]      modulation m, or logits when softmax_flag = 1
+ *   out    [N][Ho][Wo][C]
+ *   Ho = (H + 2*pad - dil*(kh - 1) - 1) / stride + 1, Wo likewise with W, kw.
+ *
+ * Limits: H, W, kh, kw, stride, dil <= 65536; one image of x and of out below
+ * 2^31 bytes (DCN_ERR_UNSUPPORTED otherwise).  N = 0 launches nothing and
+ * returns DCN_OK.  Offsets may be any value: a tap whose corners all fall
+ * outside the map, however far, contributes 0; a NaN offset makes its tap
+ * contribute 0.  Non-finite x or mask values give unspecified (but never
+ * trapping) results.
+ * Errors: DCN_ERR_INVALID_ARG for N < 0, any other dimension <= 0 (pad < 0),
+ * C % G != 0, Ho or Wo <= 0, softmax_flag not 0/1, an unknown dtype, a null
+ * pointer (N > 0) or out overlapping an input; DCN_ERR_MISALIGNED when a
+ * pointer is not aligned to the element size.
+ */
+DCN_API int dcn_forward(const void* x, const void* offset, const void* mask, void* out,
+                int N, int H, int W, int C, int G, int kh, int kw,
+                int stride, int pad, int dil, int softmax_flag, int dtype,
+                void* stream);
+
+/*
+ * msda_forward - multi-scale deformable attention core, forward.
+ *
+ * Defined by "Deformable DETR: Learn Where to Read", "A learned location can
+ * fall between cells" (x = u W_l - 1/2, y = v H_l - 1/2, bilinear tent weights
+ * over the four floor/ceil neighbours, zero outside, no clamping, no
+ * renormalisation) and "Mix samples with a per-head budget" (h_m = sum over
+ * levels l and points k of A_mlk times the sample, heads concatenated before
+ * the output projection, which is not part of this call):
+ *
+ *   out[n][q][h*D + c] = sum_{l < L, k < K} attn_w[n][q][h][l][k] *
+ *                        S_l(value[n][start_l + .][h][c], sampling_loc[n][q][h][l][k])
+ *
+ * Layouts:
+ *   value          [N][S][M][D]       levels concatenated row-major, level l at
+ *                                     rows [start_l, start_l + H_l W_l)
+ *   spatial_shapes [L][2] int64       (H_l, W_l), DEVICE memory
+ *   level_start    [L]    int64       start_l, DEVICE memory
+ *   sampling_loc   [N][Lq][M][L][K][2] normalised (u, v) = (x, y), any real value
+ *   attn_w         [N][Lq][M][L][K]   already normalised weights (used as given)
+ *   out            [N][Lq][M*D]
+ *   S is taken as level_start[L-1] + H_{L-1} * W_{L-1} (levels stored in order,
+ *   without gaps).
+ *
+ * The device contents of spatial_shapes and level_start are a precondition
+ * (positive shapes, starts inside value); they are not validated, because that
+ * would need a synchronisation.
+ * Limits: L <= 16, K <= 64, M * D and one batch item of value and out below
+ * 2^31 bytes (DCN_ERR_UNSUPPORTED otherwise).  N = 0 or Lq = 0 launches nothing
+ * and returns DCN_OK.
+ * Errors: DCN_ERR_INVALID_ARG for N < 0, Lq < 0, M, D, L or K <= 0, an unknown
+ * dtype, a null pointer (N * Lq > 0) or out overlapping an input;
+ * DCN_ERR_MISALIGNED when a pointer is not aligned to its element size.
+ */
+DCN_API int msda_forward(const void* value, const int64_t* spatial_shapes,
+                 const int64_t* level_start, const void* sampling_loc,
+                 const void* attn_w, void* out, int N, int Lq, int M, int D,
+                 int L, int K, int dtype, void* stream);
+
+/* Output size of the deformable window: (in + 2 pad - dil (k - 1) - 1) / stride + 1,
+ * or a value <= 0 when the window does not fit. */
+DCN_API int dcn_output_size(int in, int k, int stride, int pad, int dil);
+
+/* Static English text for a dcn_status_t value (never NULL). */
+DCN_API const char* dcn_status_string(int status);
+
+/* The cudaError_t of the most recent DCN_ERR_CUDA in the calling thread (0 if none). */
+DCN_API int dcn_last_cuda_error(void);
+
+/* Number of kernels this library has launched in this process (all threads). */
+DCN_API uint64_t dcn_launch_count(void);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+DCN_API int dcn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCN_B200_H */

@@ -1,0 +1,138 @@
+"""The C interface without a GPU: the library builds, loads and exports every
+symbol include/dcn.h declares, and host-side validation returns the documented
+status before any CUDA call (fake, never-dereferenced pointer values)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import deformable_attention_sampling_b200 as dcnb
+from deformable_attention_sampling_b200 import build as dcn_build
+import oracle
+
+HEADER = os.path.join(dcn_build.INCLUDE, "dcn.h")
+
+# plausible, 256-byte aligned fake device addresses; validation never reads them
+X, OFF, MASK, OUT = 0x7F0000000000, 0x7F0010000000, 0x7F0020000000, 0x7F0030000000
+F16 = 1
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dcn_build.build()
+    return dcnb.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return set(re.findall(r"^\s*DCN_API\s+(?:const\s+)?\w+\*?\s+\*?(\w+)\s*\(", text, flags=re.M))
+
+
+def test_header_declares_the_interface():
+    names = declared_functions()
+    assert {"dcn_forward", "msda_forward", "dcn_status_string"} <= names
+    assert names == set(dcnb.SIGNATURES), "binding signatures out of sync with dcn.h"
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    # the library is the in-tree build, not an installed copy
+    assert os.path.dirname(dcnb.LIB_PATH).startswith(os.path.dirname(dcn_build.LIB_DIR))
+
+
+def test_status_strings_and_version(lib):
+    assert dcnb.dcn_status_string(0) == "ok"
+    for s in (-1, -2, -3, -4, 123):
+        assert isinstance(dcnb.dcn_status_string(s), str) and dcnb.dcn_status_string(s)
+    assert dcnb.dcn_version() >= 10000
+    assert dcnb.dcn_last_cuda_error() == 0
+    assert dcnb.dcn_launch_count() == 0
+
+
+@pytest.mark.parametrize("n_in,k,stride,pad,dil", [
+    (56, 3, 1, 1, 1), (7, 3, 2, 1, 1), (10, 5, 1, 2, 2), (4, 3, 1, 0, 2), (1, 1, 1, 0, 1),
+    (3, 5, 1, 0, 1), (200, 3, 2, 0, 3)])
+def test_output_size_matches_the_oracle(lib, n_in, k, stride, pad, dil):
+    expect = oracle.out_size(n_in, k, stride, pad, dil)
+    assert dcnb.dcn_output_size(n_in, k, stride, pad, dil) == max(expect, 0)
+
+
+def call_dcn(lib, **kw):
+    args = dict(x=X, offset=OFF, mask=MASK, out=OUT, N=2, H=8, W=8, C=16, G=2, kh=3, kw=3,
+                stride=1, pad=1, dil=1, softmax_flag=0, dtype=F16, stream=None)
+    args.update(kw)
+    return lib.dcn_forward(args["x"], args["offset"], args["mask"], args["out"], args["N"],
+                           args["H"], args["W"], args["C"], args["G"], args["kh"], args["kw"],
+                           args["stride"], args["pad"], args["dil"], args["softmax_flag"],
+                           args["dtype"], args["stream"])
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(dtype=7), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(N=-1), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(H=0), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(C=15), dcnb.DCN_ERR_INVALID_ARG),            # C % G != 0
+    (dict(G=0), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(kh=0), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(stride=0), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(pad=-1), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(dil=0), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(softmax_flag=2), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(H=2, pad=0), dcnb.DCN_ERR_INVALID_ARG),      # Ho <= 0
+    (dict(x=None), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(out=None), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(out=X), dcnb.DCN_ERR_INVALID_ARG),           # out aliases x
+    (dict(out=OFF + 64), dcnb.DCN_ERR_INVALID_ARG),    # out overlaps offset
+    (dict(x=X + 1), dcnb.DCN_ERR_MISALIGNED),          # not 2-byte aligned
+    (dict(mask=MASK + 2, dtype=0), dcnb.DCN_ERR_MISALIGNED),   # f32 needs 4 bytes
+    (dict(H=70000), dcnb.DCN_ERR_UNSUPPORTED),
+    (dict(kh=33, kw=33, pad=16), dcnb.DCN_ERR_UNSUPPORTED),   # K > 1024
+    (dict(N=0), dcnb.DCN_OK),                          # nothing to do, nothing launched
+    (dict(N=0, x=None, out=None), dcnb.DCN_OK),
+])
+def test_dcn_forward_validation(lib, change, status):
+    before = dcnb.dcn_launch_count()
+    assert call_dcn(lib, **change) == status
+    assert dcnb.dcn_launch_count() == before
+
+
+def call_msda(lib, **kw):
+    args = dict(value=X, shapes=OFF, starts=OFF + 1024, loc=MASK, attn=MASK + 2 ** 24, out=OUT,
+                N=2, Lq=100, M=8, D=32, L=4, K=4, dtype=0, stream=None)
+    args.update(kw)
+    return lib.msda_forward(args["value"], args["shapes"], args["starts"], args["loc"],
+                            args["attn"], args["out"], args["N"], args["Lq"], args["M"],
+                            args["D"], args["L"], args["K"], args["dtype"], args["stream"])
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(dtype=3), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(M=0), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(D=-4), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(L=0), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(K=0), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(Lq=-1), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(L=17), dcnb.DCN_ERR_UNSUPPORTED),
+    (dict(K=65), dcnb.DCN_ERR_UNSUPPORTED),
+    (dict(shapes=None), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(out=MASK), dcnb.DCN_ERR_INVALID_ARG),        # out aliases loc
+    (dict(out=X), dcnb.DCN_ERR_INVALID_ARG),           # out aliases value
+    (dict(loc=MASK + 2), dcnb.DCN_ERR_MISALIGNED),     # f32 needs 4 bytes
+    (dict(starts=OFF + 1028), dcnb.DCN_ERR_MISALIGNED),  # int64 needs 8 bytes
+    (dict(Lq=0), dcnb.DCN_OK),
+    (dict(N=0, value=None), dcnb.DCN_OK),
+])
+def test_msda_forward_validation(lib, change, status):
+    before = dcnb.dcn_launch_count()
+    assert call_msda(lib, **change) == status
+    assert dcnb.dcn_launch_count() == before
+
+
+def test_binding_raises_with_status(lib):
+    with pytest.raises(dcnb.DcnError) as e:
+        dcnb.dcn_forward(X, OFF, MASK, OUT, 1, 4, 4, 6, 4, 3, 3, 1, 1, 1, 0, F16, stream=0)
+    assert e.value.status == dcnb.DCN_ERR_INVALID_ARG
+    assert "invalid argument" in str(e.value)
