@@ -292,12 +292,8 @@ def setup_distributed():
 
 
 def max_over_ranks(x, world, device):
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from deformable_attention_sampling_b200.sharding import max_over_ranks as reduce_max
+    return reduce_max(x, device) if world > 1 else x
 
 
 def barrier(world, device):

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <mutex>
 
 #include "dcn.h"
@@ -56,13 +57,21 @@ bool overlaps(const void* a, long long abytes, const void* b, long long bbytes) 
 }
 
 // Grid size: one resident wave of CTAs (SM count x CTAs per SM), or fewer
-// when there are fewer blocks; each CTA then strides over the blocks.
+// when there are fewer work units; each CTA then takes a contiguous share.
+//
+// The first time a kernel runs on a device with a given shared-memory size,
+// its preferred shared-memory carveout is set to what its resident CTAs need
+// (the rest of the SM's 256 KB array stays L1, which the gathers live in);
+// the carveout of a kernel only ever grows, so no earlier configuration loses
+// occupancy.
 struct GridCacheEntry {
     const void* fn;
     int device;
+    int threads;
     int smem;
     int ctas_per_sm;
     int sms;
+    int carveout;
 };
 std::mutex g_grid_mutex;
 GridCacheEntry g_grid_cache[64];
@@ -71,21 +80,45 @@ int g_grid_cache_n = 0;
 int wave_size(const void* fn, int threads, int smem) {
     int device = 0;
     if (cudaGetDevice(&device) != cudaSuccess) return 0;
-    {
-        std::lock_guard<std::mutex> lock(g_grid_mutex);
-        for (int i = 0; i < g_grid_cache_n; ++i) {
-            const GridCacheEntry& e = g_grid_cache[i];
-            if (e.fn == fn && e.device == device && e.smem == smem) return e.ctas_per_sm * e.sms;
+    std::lock_guard<std::mutex> lock(g_grid_mutex);
+    int carve_set = -1;
+    for (int i = 0; i < g_grid_cache_n; ++i) {
+        const GridCacheEntry& e = g_grid_cache[i];
+        if (e.fn == fn && e.device == device) {
+            if (e.smem == smem && e.threads == threads) return e.ctas_per_sm * e.sms;
+            if (e.carveout > carve_set) carve_set = e.carveout;
         }
     }
-    int sms = 0, per_sm = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    int sms = 0, smem_sm = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, device) !=
+            cudaSuccess)
         return 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem) != cudaSuccess)
         return 0;
     if (per_sm < 1) per_sm = 1;
-    std::lock_guard<std::mutex> lock(g_grid_mutex);
-    if (g_grid_cache_n < 64) g_grid_cache[g_grid_cache_n++] = {fn, device, smem, per_sm, sms};
+    // shared memory the resident CTAs need (1 KB per CTA is reserved by the system)
+    const long long need = (long long)per_sm * (smem + 1024);
+    int carve = smem_sm > 0 ? (int)((need * 100 + smem_sm - 1) / smem_sm) : -1;
+    if (carve > 100) carve = 100;
+    if (carve < carve_set) carve = carve_set;
+    if (carve >= 0 &&
+        cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, carve) ==
+            cudaSuccess) {
+        int per_sm2 = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm2, fn, threads, smem) !=
+                cudaSuccess || per_sm2 < per_sm) {
+            (void)cudaGetLastError();
+            (void)cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       cudaSharedmemCarveoutDefault);
+            carve = -1;
+        }
+    } else {
+        (void)cudaGetLastError();
+        carve = -1;
+    }
+    if (g_grid_cache_n < 64)
+        g_grid_cache[g_grid_cache_n++] = {fn, device, threads, smem, per_sm, sms, carve};
     return per_sm * sms;
 }
 
@@ -112,28 +145,73 @@ int launch(const void* fn, const Args& args, int num_blocks, int threads, int sm
 
 // ---------------------------------------------------------------- DCN ------
 
-template <typename T, int VB>
-const void* dcn_kernel_for(int kh, int kw, int softmax) {
-    using namespace dcnb;
-    if (kh == 3 && kw == 3) {
-        return softmax ? (const void*)dcn_fwd_kernel<T, VB, 3, 3, true>
-                       : (const void*)dcn_fwd_kernel<T, VB, 3, 3, false>;
+// Tile shape of the DCN kernel: tile_h output rows x tile_w warp runs, one
+// warp per run, at most kDcnMaxWarps warps per CTA.  A CTA sweeps its tiles
+// along the row, so its L1 footprint is its band's input rows (tile rows plus
+// the window and offset halo) times a sliding column window; the SM's L1 only
+// holds the footprint of about one such band.  The choice minimises the
+// product of
+//   - padded work      (rows and runs beyond the map in the last tiles),
+//   - vertical overfetch ((tile_h + halo) / tile_h input rows per output row),
+//   - the tail         (the last wave of tiles only partly fills the SMs),
+//   - latency exposure (fewer resident warps cover less gather latency).
+// On small maps (at most kSmallMapRows output rows) a band of the image fits
+// in L1 whatever the tile, and measured time is set by resident warps: there
+// tiles are capped at 8 warps so that three CTAs share an SM.  On larger maps
+// L1 reuse dominates and tiles grow up to kDcnMaxWarps rows (one CTA per SM).
+struct TileShape {
+    int h, w;
+};
+
+constexpr int kSmallMapRows = 64;
+
+TileShape choose_tile(int N, int Ho, int runs, int kernel_extent, int sms) {
+    constexpr int kWarpsPerSmByRegs = 25;   // 80 registers per thread
+    const int max_warps = Ho <= kSmallMapRows ? 8 : dcnb::kDcnMaxWarps;
+    const double halo = kernel_extent + 2.0 * dcnb::kPrefetchMargin;
+    TileShape best{1, 1};
+    double best_cost = 1e300;
+    for (int h = 1; h <= max_warps && h <= Ho; ++h) {
+        for (int w = 1; h * w <= max_warps && w <= runs; ++w) {
+            const int warps = h * w;
+            if (warps < 8 && warps < Ho * runs) continue;
+            const long long bands = (Ho + h - 1) / h, tx = (runs + w - 1) / w;
+            const double pad_work = (double)(bands * h * tx * w) / ((double)Ho * runs);
+            const double overfetch = (h + halo) / h;
+            int ctas = kWarpsPerSmByRegs / warps;
+            if (ctas < 1) ctas = 1;
+            const double per_slot = (double)N * bands * tx / ((double)sms * ctas);
+            const double tail = (per_slot < 1.0 ? 1.0 : std::ceil(per_slot)) / per_slot;
+            const int resident = warps * ctas < 24 ? warps * ctas : 24;
+            const double latency = 1.0 + 8.0 / resident;
+            const double cost = pad_work * overfetch * tail * latency;
+            if (cost < best_cost) {
+                best_cost = cost;
+                best = TileShape{h, w};
+            }
+        }
     }
-    return softmax ? (const void*)dcn_fwd_kernel<T, VB, 0, 0, true>
-                   : (const void*)dcn_fwd_kernel<T, VB, 0, 0, false>;
+    return best;
+}
+
+template <typename T, int VB>
+const void* dcn_kernel_for(int softmax) {
+    using namespace dcnb;
+    return softmax ? (const void*)dcn_fwd_kernel<T, VB, true>
+                   : (const void*)dcn_fwd_kernel<T, VB, false>;
 }
 
 template <typename T>
 const void* dcn_kernel_vb(int vb, int kh, int kw, int softmax) {
     switch (vb) {
-        case 32: return dcn_kernel_for<T, 32>(kh, kw, softmax);
-        case 16: return dcn_kernel_for<T, 16>(kh, kw, softmax);
-        case 8: return dcn_kernel_for<T, 8>(kh, kw, softmax);
-        case 4: return dcn_kernel_for<T, 4>(kh, kw, softmax);
+        case 32: return dcn_kernel_for<T, 32>(softmax);
+        case 16: return dcn_kernel_for<T, 16>(softmax);
+        case 8: return dcn_kernel_for<T, 8>(softmax);
+        case 4: return dcn_kernel_for<T, 4>(softmax);
         default: break;
     }
     if constexpr (sizeof(T) == 2) {
-        if (vb == 2) return dcn_kernel_for<T, 2>(kh, kw, softmax);
+        if (vb == 2) return dcn_kernel_for<T, 2>(softmax);
     }
     return nullptr;
 }
@@ -204,13 +282,32 @@ int dcn_forward(const void* x, const void* offset, const void* mask, void* out, 
     if (vb == 0) return DCN_ERR_MISALIGNED;
     const int cpt = vb / es;
     const int tpi = D / cpt;
-    if (tpi > dcnb::kDcnThreads) return DCN_ERR_UNSUPPORTED;
-    int items_per_cta = dcnb::kDcnThreads / tpi;
-    const int per_item_stage = K * 3 * es;
-    if (items_per_cta * per_item_stage + 32 > kMaxStageBytes)
-        items_per_cta = (kMaxStageBytes - 32) / per_item_stage;
-    if (items_per_cta < 1) return DCN_ERR_UNSUPPORTED;
-    const int smem = ((items_per_cta * K * 2 * es + 15) & ~15) + items_per_cta * K * es;
+    if (tpi > 32) return DCN_ERR_UNSUPPORTED;   // one item must fit in a warp
+    const int run_items = 32 / tpi;
+    const int row_items = Wo * G;
+    const int runs_per_row = (row_items + run_items - 1) / run_items;
+    int sms = 148;
+    {
+        int device = 0;
+        if (cudaGetDevice(&device) == cudaSuccess)
+            (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+        (void)cudaGetLastError();
+    }
+    const TileShape ts = choose_tile(N, Ho, runs_per_row, kh * dil, sms);
+    const int warps = ts.h * ts.w;
+    const int tiles_x = (runs_per_row + ts.w - 1) / ts.w;
+    const long long tiles_per_image = (long long)((Ho + ts.h - 1) / ts.h) * tiles_x;
+    const long long num_tiles = tiles_per_image * N;
+    if (num_tiles > kInt31) return DCN_ERR_UNSUPPORTED;
+    // per-warp shared slice for the run's offsets and masks; unstaged when the
+    // CTA's slices would not fit in the default shared-memory window
+    int stage_elems = run_items * K;
+    const int slice = ((2 * stage_elems * es + 15) & ~15) + ((stage_elems * es + 15) & ~15);
+    int smem = slice * warps;
+    if (smem > kMaxStageBytes) {
+        stage_elems = 0;
+        smem = 0;
+    }
 
     dcnb::DcnArgs a;
     a.x = x;
@@ -231,13 +328,20 @@ int dcn_forward(const void* x, const void* offset, const void* mask, void* out, 
     a.Ho = Ho;
     a.Wo = Wo;
     a.tpi = tpi;
-    a.items_per_cta = items_per_cta;
-    a.total_items = (int)items;
-    a.num_blocks = (int)((items + items_per_cta - 1) / items_per_cta);
+    a.run_items = run_items;
+    a.runs_per_row = runs_per_row;
+    a.tile_h = ts.h;
+    a.tile_w = ts.w;
+    a.tiles_x = tiles_x;
+    a.tiles_per_image = (int)tiles_per_image;
+    a.num_tiles = (int)num_tiles;
+    a.stage_elems = stage_elems;
+    a.prefetch = (((uintptr_t)x | (uintptr_t)(C * es)) % 16) == 0 ? 1 : 0;
     a.div_G = make_div((uint32_t)G);
-    a.div_Wo = make_div((uint32_t)Wo);
-    a.div_Ho = make_div((uint32_t)Ho);
     a.div_tpi = make_div((uint32_t)tpi);
+    a.div_tile_w = make_div((uint32_t)ts.w);
+    a.div_tiles_x = make_div((uint32_t)tiles_x);
+    a.div_tiles_per_image = make_div((uint32_t)tiles_per_image);
     a.pix_bytes = (uint32_t)(C * es);
     a.row_bytes = (uint32_t)((long long)W * C * es);
     a.img_bytes = img_bytes;
@@ -250,7 +354,7 @@ int dcn_forward(const void* x, const void* offset, const void* mask, void* out, 
         default: break;
     }
     if (!fn) return DCN_ERR_UNSUPPORTED;
-    return launch(fn, a, a.num_blocks, dcnb::kDcnThreads, smem, stream);
+    return launch(fn, a, a.num_tiles, 32 * warps, smem, stream);
 }
 
 int msda_forward(const void* value, const int64_t* spatial_shapes, const int64_t* level_start,

@@ -6,37 +6,43 @@
 // with zero padding outside the map and m either used as given (DCNv4) or
 // soft-maxed over the K taps of the group (DCNv3).
 //
-// Work decomposition.  A work item is one (output pixel, group) pair; items
-// are numbered pixel-major, group-minor, which is exactly the memory order of
-// the offset and mask tensors ([N,Ho,Wo,G,K,...]).  Each item is handled by
-// TPI = D / CPT threads, each owning CPT consecutive channels of the group
-// (CPT * sizeof(T) = VB bytes, at most 32: one 256-bit load per corner).
-// A block of items is therefore contiguous in offset, mask and out.
+// Work decomposition
+//   item  = one (output pixel, group) pair; items are numbered pixel-major,
+//           group-minor: the memory order of offset, mask and out.  TPI = D/CPT
+//           threads serve an item, each owning CPT consecutive channels (CPT *
+//           sizeof(T) = VB <= 32 bytes: one 256-bit load per corner).
+//   run   = 32/TPI consecutive items of one output row, served by one warp.  A
+//           run is contiguous in offset, mask and out.
+//   tile  = kDcnWarps runs at the same position in consecutive output rows.  A
+//           CTA sweeps a contiguous range of tiles, ordered along the row, so
+//           its gathers reuse the L1 lines its neighbours brought in.
 //
-//   1. The CTA copies its block's offsets and masks (one contiguous span each)
-//      into shared memory with coalesced 16-byte loads: every value is read
-//      from HBM once and each thread then reads its own item's K triples.
-//   2. Per tap, the thread splits the offset into integer and fractional parts
-//      (floor(d), d - floor(d): exact for 16-bit inputs), forms the four
-//      corner weights (1-a)(1-b)m, a(1-b)m, (1-a)b m, ab m once for its CPT
-//      channels, zeroes the weight of every corner outside the map and issues
-//      one predicated vector load per in-bounds corner.  A corner outside the
-//      map is never loaded: its registers keep the previous (finite) data and
-//      its weight is zero.
-//   3. The CPT channels accumulate in float32 with packed FFMA2; the result is
-//      rounded once to T and written with one streaming vector store.
+// Per run the warp copies the run's offsets and masks (two contiguous spans)
+// into its own slice of shared memory with coalesced 16-byte loads and then
+// syncs only itself; there is no CTA-wide barrier.  Per tap a thread splits
+// the offset into floor and fraction (exact for 16-bit inputs), forms per-axis
+// weights that are zero for corners outside the map, and issues four
+// unconditional vector loads whose coordinates are clamped into the map (a
+// clamped corner has weight 0, so its data never contributes).  One warp of
+// each CTA bulk-prefetches into L2 the x rows of the CTA's next tiles, so that
+// the gathers' L1 misses find their data in L2 instead of HBM.
+// Channels accumulate in float32 with packed FFMA2; the result is rounded once
+// and stored with one streaming vector store.
+//
 // No tensor cores: the work is a gather and a weighted sum, not a contraction.
+// The binding limit is the SM's L1 data path for scattered 32-byte gathers.
 #pragma once
 
 #include "common.cuh"
 
 namespace dcnb {
 
-constexpr int kDcnThreads = 128;
-// Offsets are clamped to +-kBigCoord before the integer conversion; any tap
-// that far out has all four corners outside every supported map (H, W <= 2^16),
-// and a NaN offset maps to -kBigCoord (fminf/fmaxf return the non-NaN operand).
-constexpr float kBigCoord = 4194304.0f;   // 2^22
+constexpr int kDcnMaxWarps = 24;             // warps per CTA = runs per tile, at most
+constexpr int kDcnMaxThreads = 32 * kDcnMaxWarps;
+// Offset floors are clamped to +-kBigCoord before the integer conversion; a
+// tap that far out has all four corners outside every supported map
+// (H, W <= 2^16), and fminf / fmaxf map a NaN offset to the bound.
+constexpr float kBigCoord = 4194304.0f;      // 2^22
 
 struct DcnArgs {
     const void* x;
@@ -47,56 +53,210 @@ struct DcnArgs {
     int kh, kw, K;
     int stride, pad, dil;
     int Ho, Wo;
-    int tpi;              // threads per item
-    int items_per_cta;    // items staged and computed per block
-    int total_items;      // N * Ho * Wo * G   (< 2^31)
-    int num_blocks;       // ceil(total_items / items_per_cta)
-    FastDiv div_G, div_Wo, div_Ho, div_tpi;
-    uint32_t pix_bytes;   // C * sizeof(T): byte stride between neighbouring pixels
-    uint32_t row_bytes;   // W * C * sizeof(T)
-    long long img_bytes;  // H * W * C * sizeof(T)
+    int tpi;                  // threads per item
+    int run_items;            // items per warp run (32 / tpi)
+    int runs_per_row;         // ceil(Wo * G / run_items)
+    int tile_h;               // output rows per tile
+    int tile_w;               // runs per tile row; the CTA has tile_h * tile_w warps
+    int tiles_x;              // ceil(runs_per_row / tile_w)
+    int tiles_per_image;      // ceil(Ho / tile_h) * tiles_x
+    int num_tiles;            // N * tiles_per_image
+    int stage_elems;          // staged mask elements per warp (run_items * K); 0 = unstaged
+    int prefetch;             // 1: bulk-prefetch upcoming tiles' x rows into L2
+    FastDiv div_G, div_tpi, div_tile_w, div_tiles_x, div_tiles_per_image;
+    uint32_t pix_bytes;       // C * sizeof(T): byte stride between neighbouring pixels
+    uint32_t row_bytes;       // W * C * sizeof(T)
+    long long img_bytes;      // H * W * C * sizeof(T)
 };
 
-// KH, KW: compile-time window (0 = runtime a.kh / a.kw).
-template <typename T, int VB, int KH, int KW, bool SOFTMAX>
-__global__ void __launch_bounds__(kDcnThreads, 4) dcn_fwd_kernel(const DcnArgs a) {
+// Copy `elems` elements of T from global `src` to shared `dst` with the lanes
+// of one warp (widest access the addresses and size allow; streaming loads).
+template <typename T>
+__device__ __forceinline__ void warp_stage(T* dst, const T* src, int elems, int lane) {
+    const int nbytes = elems * (int)sizeof(T);
+    const uintptr_t a = (uintptr_t)src | (uintptr_t)dst | (uintptr_t)nbytes;
+    if ((a & 15) == 0) {
+        const uint4* s = reinterpret_cast<const uint4*>(src);
+        uint4* d = reinterpret_cast<uint4*>(dst);
+        for (int i = lane; i < (nbytes >> 4); i += 32) {
+            uint4 v;
+            asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(s + i));
+            d[i] = v;
+        }
+    } else if ((a & 7) == 0) {
+        const uint2* s = reinterpret_cast<const uint2*>(src);
+        uint2* d = reinterpret_cast<uint2*>(dst);
+        for (int i = lane; i < (nbytes >> 3); i += 32) {
+            uint2 v;
+            asm("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                : "=r"(v.x), "=r"(v.y) : "l"(s + i));
+            d[i] = v;
+        }
+    } else if ((a & 3) == 0) {
+        const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
+        uint32_t* d = reinterpret_cast<uint32_t*>(dst);
+        for (int i = lane; i < (nbytes >> 2); i += 32) d[i] = __ldg(s + i);
+    } else {
+        const unsigned short* s = reinterpret_cast<const unsigned short*>(src);
+        unsigned short* d = reinterpret_cast<unsigned short*>(dst);
+        for (int i = lane; i < (nbytes >> 1); i += 32) d[i] = __ldg(s + i);
+    }
+}
+
+// Tiles ahead of the current one whose x rows are prefetched into L2, and the
+// margin (pixels) added around a tile's undeformed window for the offsets.
+constexpr int kPrefetchAhead = 2;
+constexpr int kPrefetchMargin = 4;
+
+// A tile's batch item, first output row and first run (tiles are numbered
+// image-major, then band of tile_h rows, then tile_w runs along the row).
+struct TileCoord {
+    int n, oy0, run0;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const DcnArgs& a, int tile) {
+    const int n = (int)a.div_tiles_per_image.div((uint32_t)tile);
+    const int rem = tile - n * a.tiles_per_image;
+    const int band = (int)a.div_tiles_x.div((uint32_t)rem);
+    const int tx = rem - band * a.tiles_x;
+    return TileCoord{n, band * a.tile_h, tx * a.tile_w};
+}
+
+// Bulk-prefetch into L2 the rows of x that `tile` gathers from (its output
+// rows' window plus a margin for the offsets), one contiguous span per input
+// row, issued by the lanes of one warp.  A prefetch is only a hint: it moves
+// no data into the kernel and changes no result.  Requires 16-byte aligned
+// x rows and pixels (checked on the host).
+__device__ __forceinline__ void prefetch_tile_x(const DcnArgs& a, int tile, int lane) {
+    if (tile >= a.num_tiles) return;
+    const TileCoord tc = decode_tile(a, tile);
+    const int n = tc.n;
+    const int oy0 = tc.oy0;
+    const int oy1 = min(oy0 + a.tile_h, a.Ho) - 1;
+    const int i0 = tc.run0 * a.run_items;
+    const int i1 = min(i0 + a.tile_w * a.run_items, a.Wo * a.G) - 1;
+    const int ox0 = (int)a.div_G.div((uint32_t)i0), ox1 = (int)a.div_G.div((uint32_t)i1);
+    const int y_lo = max(oy0 * a.stride - a.pad - kPrefetchMargin, 0);
+    const int y_hi = min(oy1 * a.stride - a.pad + (a.kh - 1) * a.dil + kPrefetchMargin, a.H - 1);
+    const int x_lo = max(ox0 * a.stride - a.pad - kPrefetchMargin, 0);
+    const int x_hi = min(ox1 * a.stride - a.pad + (a.kw - 1) * a.dil + kPrefetchMargin, a.W - 1);
+    if (y_lo > y_hi || x_lo > x_hi) return;
+    const uint32_t span = (uint32_t)(x_hi - x_lo + 1) * a.pix_bytes;
+    const char* base = static_cast<const char*>(a.x) + (long long)n * a.img_bytes +
+                       (long long)x_lo * a.pix_bytes;
+    for (int y = y_lo + lane; y <= y_hi; y += 32) {
+        const char* p = base + (long long)y * a.row_bytes;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(span)
+                     : "memory");
+    }
+}
+
+// One tap of one item: the four corner weights (zero for a corner outside the
+// map) and the byte offsets, within the image, of the four corners to load
+// (coordinates clamped into the map, so every load is in bounds).
+struct TapGeom {
+    uint32_t off[4];
+    float w[4];
+};
+
+__device__ __forceinline__ TapGeom tap_geometry(const DcnArgs& a, int bxk, int byk, float dx,
+                                                float dy, float m) {
+    TapGeom t;
+    float fx = floorf(dx), fy = floorf(dy);
+    const float ax = dx - fx, ay = dy - fy;
+    fx = fminf(fmaxf(fx, -kBigCoord), kBigCoord);
+    fy = fminf(fmaxf(fy, -kBigCoord), kBigCoord);
+    const int x0 = bxk + (int)fx, y0 = byk + (int)fy;
+    const int x1 = x0 + 1, y1 = y0 + 1;
+    const bool vx0 = (unsigned)x0 < (unsigned)a.W, vx1 = (unsigned)x1 < (unsigned)a.W;
+    const bool vy0 = (unsigned)y0 < (unsigned)a.H, vy1 = (unsigned)y1 < (unsigned)a.H;
+    // per-axis weights, zero for a corner outside the map
+    const float wx0 = vx0 ? 1.f - ax : 0.f, wx1 = vx1 ? ax : 0.f;
+    const float wy0 = vy0 ? (1.f - ay) * m : 0.f, wy1 = vy1 ? ay * m : 0.f;
+    t.w[0] = wx0 * wy0;
+    t.w[1] = wx1 * wy0;
+    t.w[2] = wx0 * wy1;
+    t.w[3] = wx1 * wy1;
+    // coordinates clamped into the map: every load is in bounds
+    const uint32_t cx0 = vx0 ? (uint32_t)x0 : 0u, cx1 = vx1 ? (uint32_t)x1 : 0u;
+    const uint32_t cy0 = vy0 ? (uint32_t)y0 : 0u, cy1 = vy1 ? (uint32_t)y1 : 0u;
+    const uint32_t r0 = cy0 * a.row_bytes, r1 = cy1 * a.row_bytes;
+    const uint32_t c0 = cx0 * a.pix_bytes, c1 = cx1 * a.pix_bytes;
+    t.off[0] = r0 + c0;
+    t.off[1] = r0 + c1;
+    t.off[2] = r1 + c0;
+    t.off[3] = r1 + c1;
+    return t;
+}
+
+template <typename T, int VB, bool SOFTMAX>
+__global__ void __launch_bounds__(kDcnMaxThreads, 1) dcn_fwd_kernel(const DcnArgs a) {
     constexpr int CPT = VB / (int)sizeof(T);
     constexpr int NW = VB >= 4 ? VB / 4 : 1;
     extern __shared__ __align__(16) unsigned char smem[];
 
-    const int kh = KH ? KH : a.kh;
-    const int kw = KW ? KW : a.kw;
+    const int kh = a.kh;
+    const int kw = a.kw;
     const int K = kh * kw;
-    T* s_off = reinterpret_cast<T*>(smem);
-    const int off_span = ((a.items_per_cta * K * 2 * (int)sizeof(T)) + 15) & ~15;
-    T* s_mask = reinterpret_cast<T*>(smem + off_span);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const bool staged = a.stage_elems > 0;
+    // this warp's slice of shared memory: offsets, then masks
+    const int off_slice = ((2 * a.stage_elems * (int)sizeof(T)) + 15) & ~15;
+    const int slice = off_slice + ((a.stage_elems * (int)sizeof(T) + 15) & ~15);
+    T* s_off = reinterpret_cast<T*>(smem + warp * slice);
+    T* s_mask = reinterpret_cast<T*>(smem + warp * slice + off_slice);
 
-    const int li = (int)a.div_tpi.div(threadIdx.x);          // item within the block
-    const int chunk = (int)threadIdx.x - li * a.tpi;          // channel chunk of the item
+    const int li = (int)a.div_tpi.div((uint32_t)lane);     // item within the run
+    const int chunk = lane - li * a.tpi;                    // channel chunk of the item
+    const int row_items = a.Wo * a.G;
+    const int warp_row = (int)a.div_tile_w.div((uint32_t)warp);   // this warp's row in a tile
+    const int warp_col = warp - warp_row * a.tile_w;               // and its run
 
-    for (int blk = blockIdx.x; blk < a.num_blocks; blk += gridDim.x) {
-        const int item0 = blk * a.items_per_cta;
-        const int nitems = min(a.items_per_cta, a.total_items - item0);
-        __syncthreads();   // the previous block's shared reads are complete
-        stage_span(s_off, static_cast<const T*>(a.offset) + (long long)item0 * K * 2,
-                   nitems * K * 2 * (int)sizeof(T));
-        stage_span(s_mask, static_cast<const T*>(a.mask) + (long long)item0 * K,
-                   nitems * K * (int)sizeof(T));
-        __syncthreads();
+    // contiguous, balanced range of tiles for this CTA
+    const int t_begin = (int)(((long long)a.num_tiles * blockIdx.x) / gridDim.x);
+    const int t_end = (int)(((long long)a.num_tiles * (blockIdx.x + 1)) / gridDim.x);
+
+    if (a.prefetch && warp == 0) {
+        for (int t = t_begin; t < min(t_begin + kPrefetchAhead, t_end); ++t)
+            prefetch_tile_x(a, t, lane);
+    }
+
+    for (int tile = t_begin; tile < t_end; ++tile) {
+        if (a.prefetch && warp == 0 && tile + kPrefetchAhead < t_end)
+            prefetch_tile_x(a, tile + kPrefetchAhead, lane);
+        const TileCoord tc = decode_tile(a, tile);
+        const int n = tc.n;
+        const int oy = tc.oy0 + warp_row;
+        const int run = tc.run0 + warp_col;
+        if (oy >= a.Ho || run >= a.runs_per_row) continue;   // warp-uniform
+        const int i0 = run * a.run_items;                    // first item of the run in its row
+        const int nitems = min(a.run_items, row_items - i0);
+        const long long item_base = ((long long)n * a.Ho + oy) * row_items + i0;
+
+        const T* offp;
+        const T* maskp;
+        if (staged) {
+            __syncwarp();                                    // previous run's reads are done
+            warp_stage(s_off, static_cast<const T*>(a.offset) + item_base * K * 2,
+                       nitems * K * 2, lane);
+            warp_stage(s_mask, static_cast<const T*>(a.mask) + item_base * K, nitems * K,
+                       lane);
+            __syncwarp();
+            offp = s_off + li * K * 2;
+            maskp = s_mask + li * K;
+        } else {
+            offp = static_cast<const T*>(a.offset) + (item_base + li) * K * 2;
+            maskp = static_cast<const T*>(a.mask) + (item_base + li) * K;
+        }
         if (li >= nitems) continue;
 
-        const int item = item0 + li;
-        const int pix = (int)a.div_G.div((uint32_t)item);     // n*Ho*Wo + oy*Wo + ox
-        const int g = item - pix * a.G;
-        const int t = (int)a.div_Wo.div((uint32_t)pix);
-        const int ox = pix - t * a.Wo;
-        const int n = (int)a.div_Ho.div((uint32_t)t);
-        const int oy = t - n * a.Ho;
-
+        const int item_in_row = i0 + li;
+        const int ox = (int)a.div_G.div((uint32_t)item_in_row);
+        const int g = item_in_row - ox * a.G;
         const char* xb = static_cast<const char*>(a.x) + (long long)n * a.img_bytes +
                          (long long)(g * a.D + chunk * CPT) * (int)sizeof(T);
-        const T* offp = s_off + li * K * 2;
-        const T* maskp = s_mask + li * K;
         const int bx = ox * a.stride - a.pad;
         const int by = oy * a.stride - a.pad;
 
@@ -109,70 +269,66 @@ __global__ void __launch_bounds__(kDcnThreads, 4) dcn_fwd_kernel(const DcnArgs a
             for (int k = 0; k < K; ++k) s += expf(Elem<T>::one(maskp + k) - zmax);
             inv_sum = 1.f / s;
         }
+        auto modulation = [&](int k) {
+            const float z = Elem<T>::one(maskp + k);
+            if constexpr (SOFTMAX) return expf(z - zmax) * inv_sum;
+            return z;
+        };
 
         float acc[CPT];
 #pragma unroll
         for (int i = 0; i < CPT; ++i) acc[i] = 0.f;
-        uint32_t r00[NW], r01[NW], r10[NW], r11[NW];   // stale data stays finite
-#pragma unroll
-        for (int i = 0; i < NW; ++i) r00[i] = r01[i] = r10[i] = r11[i] = 0u;
 
+        // Rolling corner pipeline over the taps (k = ix * kh + iy, walked with
+        // iy fastest): the geometry of tap k+1 is computed while tap k's four
+        // loads are in flight, and each corner's registers are refilled with
+        // tap k+1's corner right after they are consumed.  Four loads stay in
+        // flight with the registers of one tap.
+        uint32_t v[4][NW];
+        float w[4];
+        int nix = 0, niy = 0;            // the next tap to prepare
+        auto geometry = [&]() {
+            const int k = nix * kh + niy;
+            float dx, dy;
+            load_pair<T>(offp + 2 * k, dx, dy);
+            const TapGeom t = tap_geometry(a, bx + nix * a.dil, by + niy * a.dil, dx, dy,
+                                           modulation(k));
+            if (++niy == kh) {
+                niy = 0;
+                ++nix;
+            }
+            return t;
+        };
+        {
+            const TapGeom t0 = geometry();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                load_vec<VB>(xb + t0.off[c], v[c]);
+                w[c] = t0.w[c];
+            }
+        }
 #pragma unroll 1
-        for (int ix = 0; ix < kw; ++ix) {
+        for (int k = 0; k < K; ++k) {
+            const bool more = k + 1 < K;
+            TapGeom tn;
+            if (more) tn = geometry();
+            float f[CPT];
 #pragma unroll
-            for (int iy = 0; iy < kh; ++iy) {
-                const int k = ix * kh + iy;
-                float dx, dy;
-                load_pair<T>(offp + 2 * k, dx, dy);
-                float m = Elem<T>::one(maskp + k);
-                if constexpr (SOFTMAX) m = expf(m - zmax) * inv_sum;
-
-                // integer and fractional parts of the offset
-                float fx = floorf(dx), fy = floorf(dy);
-                const float ax = dx - fx, ay = dy - fy;
-                fx = fminf(fmaxf(fx, -kBigCoord), kBigCoord);
-                fy = fminf(fmaxf(fy, -kBigCoord), kBigCoord);
-                const int x0 = bx + ix * a.dil + (int)fx;
-                const int y0 = by + iy * a.dil + (int)fy;
-                const bool vx0 = (unsigned)x0 < (unsigned)a.W;
-                const bool vx1 = (unsigned)(x0 + 1) < (unsigned)a.W;
-                const bool vy0 = (unsigned)y0 < (unsigned)a.H;
-                const bool vy1 = (unsigned)(y0 + 1) < (unsigned)a.H;
-
-                const float mb1 = m * ay;
-                const float mb0 = m - mb1;
-                const float w00 = (vx0 && vy0) ? (1.f - ax) * mb0 : 0.f;
-                const float w01 = (vx1 && vy0) ? ax * mb0 : 0.f;
-                const float w10 = (vx0 && vy1) ? (1.f - ax) * mb1 : 0.f;
-                const float w11 = (vx1 && vy1) ? ax * mb1 : 0.f;
-
-                // byte offsets within the image; only in-bounds corners are used,
-                // and those lie in [0, 2^31), so 32-bit wrap-around is harmless
-                const uint32_t o00 = (uint32_t)y0 * a.row_bytes + (uint32_t)x0 * a.pix_bytes;
-                const uint32_t o01 = o00 + a.pix_bytes;
-                const uint32_t o10 = o00 + a.row_bytes;
-                const uint32_t o11 = o10 + a.pix_bytes;
-                if (vx0 && vy0) load_vec<VB>(xb + (int)o00, r00);
-                if (vx1 && vy0) load_vec<VB>(xb + (int)o01, r01);
-                if (vx0 && vy1) load_vec<VB>(xb + (int)o10, r10);
-                if (vx1 && vy1) load_vec<VB>(xb + (int)o11, r11);
-
-                float f[CPT];
-                widen<T, CPT>(r00, f);
-                axpy<CPT>(acc, w00, f);
-                widen<T, CPT>(r01, f);
-                axpy<CPT>(acc, w01, f);
-                widen<T, CPT>(r10, f);
-                axpy<CPT>(acc, w10, f);
-                widen<T, CPT>(r11, f);
-                axpy<CPT>(acc, w11, f);
+            for (int c = 0; c < 4; ++c) {
+                widen<T, CPT>(v[c], f);
+                axpy<CPT>(acc, w[c], f);
+                if (more) load_vec<VB>(xb + tn.off[c], v[c]);
+            }
+            if (more) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) w[c] = tn.w[c];
             }
         }
 
         uint32_t o[NW];
         narrow<T, CPT>(acc, o);
         char* ob = static_cast<char*>(a.out) +
-                   ((long long)pix * a.C + g * a.D + chunk * CPT) * (int)sizeof(T);
+                   ((item_base + li) * a.D + chunk * CPT) * (int)sizeof(T);
         store_vec<VB>(ob, o);
     }
 }
