@@ -37,13 +37,19 @@ import gen  # noqa: E402
 
 METRIC = ("sampled taps/s & achieved HBM GB/s vs peak "
           "(DCNv4 fp16 fwd, 64×56²×64, G=4)")
-L2_BYTES = 126 * 1024 * 1024
+# Random 32-byte gathers that hit in L1 move at most this many bytes per SM
+# clock on B200 (measured with a random ld.global.nc.v8 probe, L1-resident
+# footprint; the rate falls to about 30 B/clk when the footprint spills to L2).
+L1_GATHER_BYTES_PER_CLK = 58.0
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic of the timed kernel from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum per launch, headline workload), with the hash of the
 # kernel sources it was taken on; reported as null once the sources change.
-NCU_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None}
+NCU_TRAFFIC = {
+    "source_sha256": "dbbd5eda7ae979c14fa9dde969cff6742468141b972e1367bca0742794417906",
+    "bytes_per_launch": 69166336 + 3505408,   # DRAM read + write, one headline launch
+}
 
 KERNEL_SOURCES = [
     "deformable_attention_sampling_b200/csrc/common.cuh",
@@ -157,6 +163,24 @@ class ClockSampler:
         reasons = [name for bit, name in self.REASONS.items() if mask & bit]
         return {"sm_mhz": statistics.median(s for s, _ in self.samples),
                 "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+def on_chip_roofline(w, ms_per_launch, sampler, device):
+    """The SM-side bound: every tap reads four corner vectors of D channels
+    through L1 (the kernels load all four, out-of-map ones from a clamped
+    address with zero weight).  Peak = the measured L1 gather rate x SMs x the
+    median SM clock sampled during the timed region."""
+    es = gen.DTYPES[w.dtype].itemsize
+    gathered = w.taps() * 4 * w.D * es
+    achieved = gathered / (ms_per_launch * 1e-3) / 1e9
+    clocks = sampler.summary()
+    mhz = clocks["sm_mhz"] or clocks["sm_max_mhz"] or 1965
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    peak = L1_GATHER_BYTES_PER_CLK * sms * mhz * 1e6 / 1e9
+    return {"bound": "l1_gather", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "gathered_bytes_per_launch": gathered,
+            "peak_basis": f"{L1_GATHER_BYTES_PER_CLK:g} B/clk/SM measured random 32 B gathers"
+                          f" x {sms} SMs x {mhz} MHz"}
 
 
 # ------------------------------------------------------------------ runners
@@ -316,7 +340,8 @@ def run_b200(args):
 
     runner = make_runner(w, seed=1000 + rank, device=device)
     bytes_per_step = w.compulsory_bytes()
-    n_sets = max(2, int(np.ceil(3 * L2_BYTES / bytes_per_step)))
+    l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
+    n_sets = max(2, int(np.ceil(3 * l2_bytes / bytes_per_step)))
     sets = [runner.alloc_set() for _ in range(n_sets)]
     stream = torch.cuda.current_stream(device)
     handle = int(stream.cuda_stream)
@@ -387,7 +412,7 @@ def run_b200(args):
         config = {"workload": w.name, "global_batch": w.N * world,
                   "per_gpu_batch": w.N, "dtype_storage": w.dtype, "accumulate": "f32",
                   "l2": f"{n_sets} rotating input/output sets ({n_sets * bytes_per_step / 1e6:.0f} MB"
-                        f" > L2 {L2_BYTES / 1e6:.0f} MB)",
+                        f" > 3 x L2 {l2_bytes / 1e6:.0f} MB)",
                   "parallelism": f"dp{world}" if world > 1 else "single GPU"}
         if isinstance(w, gen.DcnWorkload):
             config.update({"H": w.H, "W": w.W, "C": w.C, "G": w.G, "kernel": f"{w.kh}x{w.kw}",
@@ -417,6 +442,7 @@ def run_b200(args):
                          "kernel": kernel, "algorithmic_bytes_per_launch": bytes_per_step,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_src == "measured" else "fallback 6.65 TB/s"},
+            "on_chip": on_chip_roofline(w, ms_local / args.steps, sampler, device),
             "e2e": {"value": taps_total / (e2e_ms * 1e-3), "unit": "taps/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "steps": e2e_steps},

@@ -54,5 +54,20 @@ def build(force=False, verbose=False):
     return LIB
 
 
+PROBE_SRC = os.path.join(CSRC, "l1_gather_probe.cu")
+PROBE = os.path.join(LIB_DIR, "l1_gather_probe")
+
+
+def build_probe():
+    """Compile the gather-rate probe (a standalone program) next to the library."""
+    os.makedirs(LIB_DIR, exist_ok=True)
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
+           PROBE_SRC, "-o", PROBE]
+    subprocess.run(cmd, check=True)
+    return PROBE
+
+
 if __name__ == "__main__":
     print(build(force=True, verbose="--verbose" in sys.argv))
+    if "--probe" in sys.argv:
+        print(build_probe())

@@ -386,13 +386,17 @@ int msda_forward(const void* value, const int64_t* spatial_shapes, const int64_t
     if (vb == 0) return DCN_ERR_MISALIGNED;
     const int cpt = vb / es;
     const int tpi = D / cpt;
-    if (tpi > dcnb::kMsdaThreads) return DCN_ERR_UNSUPPORTED;
-    int items_per_cta = dcnb::kMsdaThreads / tpi;
-    const int per_item_stage = LK * 3 * es;
-    if (items_per_cta * per_item_stage + 32 > kMaxStageBytes)
-        items_per_cta = (kMaxStageBytes - 32) / per_item_stage;
-    if (items_per_cta < 1) return DCN_ERR_UNSUPPORTED;
-    const int smem = ((items_per_cta * LK * 2 * es + 15) & ~15) + items_per_cta * LK * es;
+    if (tpi > 32) return DCN_ERR_UNSUPPORTED;   // one item must fit in a warp
+    const int run_items = 32 / tpi;
+    // per-warp shared slice for the run's locations and weights; unstaged when
+    // the CTA's slices would not fit in the default shared-memory window
+    int stage_elems = run_items * LK;
+    const int slice = ((2 * stage_elems * es + 15) & ~15) + ((stage_elems * es + 15) & ~15);
+    int smem = slice * dcnb::kMsdaWarps;
+    if (smem > kMaxStageBytes) {
+        stage_elems = 0;
+        smem = 0;
+    }
 
     dcnb::MsdaArgs a;
     a.value = value;
@@ -407,9 +411,10 @@ int msda_forward(const void* value, const int64_t* spatial_shapes, const int64_t
     a.L = L;
     a.K = K;
     a.tpi = tpi;
-    a.items_per_cta = items_per_cta;
+    a.run_items = run_items;
     a.total_items = (int)items;
-    a.num_blocks = (int)((items + items_per_cta - 1) / items_per_cta);
+    a.num_runs = (int)((items + run_items - 1) / run_items);
+    a.stage_elems = stage_elems;
     a.div_M = make_div((uint32_t)M);
     a.div_Lq = make_div((uint32_t)Lq);
     a.div_tpi = make_div((uint32_t)tpi);
@@ -422,7 +427,9 @@ int msda_forward(const void* value, const int64_t* spatial_shapes, const int64_t
         default: break;
     }
     if (!fn) return DCN_ERR_UNSUPPORTED;
-    return launch(fn, a, a.num_blocks, dcnb::kMsdaThreads, smem, stream);
+    // one unit of work per warp: a CTA's warps share its range of runs
+    const int num_ctas = (a.num_runs + dcnb::kMsdaWarps - 1) / dcnb::kMsdaWarps;
+    return launch(fn, a, num_ctas, dcnb::kMsdaThreads, smem, stream);
 }
 
 const char* dcn_status_string(int status) {

@@ -6,11 +6,21 @@
 //   S_l(f, u, v): x = u W_l - 1/2, y = v H_l - 1/2; bilinear over the four
 //   floor/ceil neighbours, zero outside, no clamping, no renormalisation.
 //
-// Work decomposition mirrors the DCN kernel: a work item is one (batch,
-// query, head) triple, numbered in the memory order of loc / attn / out, and
-// TPI = D / CPT threads share it, each owning CPT consecutive channels
-// (CPT * sizeof(T) <= 32 bytes: one vector load per corner).  The CTA stages
-// its block's locations and weights (contiguous spans) into shared memory.
+// Work decomposition mirrors the DCN kernel:
+//   item = one (batch, query, head) triple, numbered in the memory order of
+//          loc, attn and out; TPI = D / CPT threads share it, each owning CPT
+//          consecutive channels (CPT * sizeof(T) <= 32 bytes: one vector load
+//          per corner).
+//   run  = 32 / TPI consecutive items served by one warp (at D = 32 fp32: the
+//          8 heads of one query).  A run is contiguous in loc, attn and out;
+//          the warp stages its run's locations and weights into its own slice
+//          of shared memory and syncs only itself.
+// Each CTA takes a contiguous range of runs.  Per item the L*K taps run as a
+// rolling corner pipeline: the next tap's geometry is computed while the
+// current tap's four loads are in flight, and each corner's registers are
+// refilled with the next tap's corner as soon as they are consumed.  Corners
+// outside the level are loaded from a clamped in-level address with zero
+// weight.
 //
 // Location arithmetic: x = u W - 1/2 is formed as hi = u*W, lo = fma(u, W, -hi)
 // (the exact rounding error of the product), x0 = floor(hi - 1/2) and
@@ -23,7 +33,8 @@
 
 namespace dcnb {
 
-constexpr int kMsdaThreads = 128;
+constexpr int kMsdaWarps = 4;
+constexpr int kMsdaThreads = 32 * kMsdaWarps;
 constexpr int kMsdaMaxLevels = 16;
 
 struct MsdaArgs {
@@ -34,10 +45,11 @@ struct MsdaArgs {
     const void* attn;
     void* out;
     int Lq, M, D, L, K;
-    int tpi;
-    int items_per_cta;
+    int tpi;                     // threads per item
+    int run_items;               // items per warp run (32 / tpi)
     int total_items;             // N * Lq * M
-    int num_blocks;
+    int num_runs;                // ceil(total_items / run_items)
+    int stage_elems;             // staged weights per warp (run_items * L * K); 0 = unstaged
     FastDiv div_M, div_Lq, div_tpi;
 };
 
@@ -61,6 +73,68 @@ __device__ __forceinline__ float level_coord(float u, float size, int* cell) {
     return a;
 }
 
+// One tap: byte offsets (from the item's value base) of the four corners to
+// load, clamped into the level, and their weights (zero outside the level).
+struct MsdaTap {
+    long long off[4];
+    float w[4];
+};
+
+__device__ __forceinline__ MsdaTap msda_tap(const int (*lvl)[3], long long pix_bytes, int l,
+                                            float u, float v, float A) {
+    MsdaTap t;
+    const int Hl = lvl[l][0], Wl = lvl[l][1];
+    int x0, y0;
+    const float ax = level_coord(u, (float)Wl, &x0);
+    const float ay = level_coord(v, (float)Hl, &y0);
+    const int x1 = x0 + 1, y1 = y0 + 1;
+    const bool vx0 = (unsigned)x0 < (unsigned)Wl, vx1 = (unsigned)x1 < (unsigned)Wl;
+    const bool vy0 = (unsigned)y0 < (unsigned)Hl, vy1 = (unsigned)y1 < (unsigned)Hl;
+    const float wx0 = vx0 ? 1.f - ax : 0.f, wx1 = vx1 ? ax : 0.f;
+    const float wy0 = vy0 ? (1.f - ay) * A : 0.f, wy1 = vy1 ? ay * A : 0.f;
+    t.w[0] = wx0 * wy0;
+    t.w[1] = wx1 * wy0;
+    t.w[2] = wx0 * wy1;
+    t.w[3] = wx1 * wy1;
+    const int cx0 = vx0 ? x0 : 0, cx1 = vx1 ? x1 : 0;
+    const int cy0 = vy0 ? y0 : 0, cy1 = vy1 ? y1 : 0;
+    // an empty level (non-positive shape) loads row 0 with zero weights
+    const long long start = (Hl > 0 && Wl > 0) ? (long long)lvl[l][2] : 0;
+    const long long row0 = start + (long long)cy0 * Wl;
+    const long long row1 = start + (long long)cy1 * Wl;
+    t.off[0] = (row0 + cx0) * pix_bytes;
+    t.off[1] = (row0 + cx1) * pix_bytes;
+    t.off[2] = (row1 + cx0) * pix_bytes;
+    t.off[3] = (row1 + cx1) * pix_bytes;
+    return t;
+}
+
+// Copy `elems` elements of T from global `src` to shared `dst` with the lanes
+// of one warp (the widest access the addresses and the size allow).
+template <typename T>
+__device__ __forceinline__ void msda_warp_stage(T* dst, const T* src, int elems, int lane) {
+    const int nbytes = elems * (int)sizeof(T);
+    const uintptr_t al = (uintptr_t)src | (uintptr_t)dst | (uintptr_t)nbytes;
+    if ((al & 15) == 0) {
+        const uint4* s = reinterpret_cast<const uint4*>(src);
+        uint4* d = reinterpret_cast<uint4*>(dst);
+        for (int i = lane; i < (nbytes >> 4); i += 32) {
+            uint4 x;
+            asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w) : "l"(s + i));
+            d[i] = x;
+        }
+    } else if ((al & 3) == 0) {
+        const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
+        uint32_t* d = reinterpret_cast<uint32_t*>(dst);
+        for (int i = lane; i < (nbytes >> 2); i += 32) d[i] = __ldg(s + i);
+    } else {
+        const unsigned short* s = reinterpret_cast<const unsigned short*>(src);
+        unsigned short* d = reinterpret_cast<unsigned short*>(dst);
+        for (int i = lane; i < (nbytes >> 1); i += 32) d[i] = __ldg(s + i);
+    }
+}
+
 template <typename T, int VB>
 __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArgs a) {
     constexpr int CPT = VB / (int)sizeof(T);
@@ -71,92 +145,100 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArg
 
     const int L = a.L, K = a.K;
     const int LK = L * K;
-    T* s_loc = reinterpret_cast<T*>(smem);
-    const int loc_span = ((a.items_per_cta * LK * 2 * (int)sizeof(T)) + 15) & ~15;
-    T* s_w = reinterpret_cast<T*>(smem + loc_span);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const bool staged = a.stage_elems > 0;
+    const int loc_slice = ((2 * a.stage_elems * (int)sizeof(T)) + 15) & ~15;
+    const int slice = loc_slice + ((a.stage_elems * (int)sizeof(T) + 15) & ~15);
+    T* s_loc = reinterpret_cast<T*>(smem + warp * slice);
+    T* s_w = reinterpret_cast<T*>(smem + warp * slice + loc_slice);
 
     if (threadIdx.x < L) {
         // a non-positive shape (a broken precondition) makes the level empty
-        // instead of turning the unsigned bounds tests below into no-ops
+        // instead of turning the unsigned bounds tests into no-ops
         s_lvl[threadIdx.x][0] = (int)max(a.shapes[2 * threadIdx.x], (int64_t)0);
         s_lvl[threadIdx.x][1] = (int)max(a.shapes[2 * threadIdx.x + 1], (int64_t)0);
         s_lvl[threadIdx.x][2] = (int)a.level_start[threadIdx.x];
     }
     if (threadIdx.x == 0)
         s_S = a.level_start[L - 1] + a.shapes[2 * (L - 1)] * a.shapes[2 * (L - 1) + 1];
+    __syncthreads();
 
-    const int li = (int)a.div_tpi.div(threadIdx.x);
-    const int chunk = (int)threadIdx.x - li * a.tpi;
+    const int li = (int)a.div_tpi.div((uint32_t)lane);   // item within the run
+    const int chunk = lane - li * a.tpi;
     const long long pix_bytes = (long long)a.M * a.D * (int)sizeof(T);   // one value row
 
-    for (int blk = blockIdx.x; blk < a.num_blocks; blk += gridDim.x) {
-        const int item0 = blk * a.items_per_cta;
-        const int nitems = min(a.items_per_cta, a.total_items - item0);
-        __syncthreads();
-        stage_span(s_loc, static_cast<const T*>(a.loc) + (long long)item0 * LK * 2,
-                   nitems * LK * 2 * (int)sizeof(T));
-        stage_span(s_w, static_cast<const T*>(a.attn) + (long long)item0 * LK,
-                   nitems * LK * (int)sizeof(T));
-        __syncthreads();
+    // contiguous, balanced range of runs for this CTA; its warps interleave
+    const int r_begin = (int)(((long long)a.num_runs * blockIdx.x) / gridDim.x);
+    const int r_end = (int)(((long long)a.num_runs * (blockIdx.x + 1)) / gridDim.x);
+
+    for (int run = r_begin + warp; run < r_end; run += kMsdaWarps) {
+        const int item0 = run * a.run_items;
+        const int nitems = min(a.run_items, a.total_items - item0);
+        const T* locp;
+        const T* wp;
+        if (staged) {
+            __syncwarp();
+            msda_warp_stage(s_loc, static_cast<const T*>(a.loc) + (long long)item0 * LK * 2,
+                            nitems * LK * 2, lane);
+            msda_warp_stage(s_w, static_cast<const T*>(a.attn) + (long long)item0 * LK,
+                            nitems * LK, lane);
+            __syncwarp();
+            locp = s_loc + li * LK * 2;
+            wp = s_w + li * LK;
+        } else {
+            locp = static_cast<const T*>(a.loc) + (long long)(item0 + li) * LK * 2;
+            wp = static_cast<const T*>(a.attn) + (long long)(item0 + li) * LK;
+        }
         if (li >= nitems) continue;
 
         const int item = item0 + li;                  // (n * Lq + q) * M + h
         const int nq = (int)a.div_M.div((uint32_t)item);
         const int h = item - nq * a.M;
         const int n = (int)a.div_Lq.div((uint32_t)nq);
-
         const char* vb = static_cast<const char*>(a.value) +
                          ((long long)n * s_S * a.M + h) * a.D * (int)sizeof(T) +
                          (long long)chunk * CPT * (int)sizeof(T);
-        const T* locp = s_loc + li * LK * 2;
-        const T* wp = s_w + li * LK;
 
         float acc[CPT];
 #pragma unroll
         for (int i = 0; i < CPT; ++i) acc[i] = 0.f;
-        uint32_t r00[NW], r01[NW], r10[NW], r11[NW];
-#pragma unroll
-        for (int i = 0; i < NW; ++i) r00[i] = r01[i] = r10[i] = r11[i] = 0u;
 
-        for (int l = 0; l < L; ++l) {
-            const int Hl = s_lvl[l][0], Wl = s_lvl[l][1];
-            const char* lb = vb + (long long)s_lvl[l][2] * pix_bytes;
-            const float Wf = (float)Wl, Hf = (float)Hl;
-#pragma unroll 2
-            for (int k = 0; k < K; ++k) {
-                const int t = l * K + k;
-                float u, v;
-                load_pair<T>(locp + 2 * t, u, v);
-                const float A = Elem<T>::one(wp + t);
-                int x0, y0;
-                const float ax = level_coord(u, Wf, &x0);
-                const float ay = level_coord(v, Hf, &y0);
-                const bool vx0 = (unsigned)x0 < (unsigned)Wl;
-                const bool vx1 = (unsigned)(x0 + 1) < (unsigned)Wl;
-                const bool vy0 = (unsigned)y0 < (unsigned)Hl;
-                const bool vy1 = (unsigned)(y0 + 1) < (unsigned)Hl;
-                const float mb1 = A * ay;
-                const float mb0 = A - mb1;
-                const float w00 = (vx0 && vy0) ? (1.f - ax) * mb0 : 0.f;
-                const float w01 = (vx1 && vy0) ? ax * mb0 : 0.f;
-                const float w10 = (vx0 && vy1) ? (1.f - ax) * mb1 : 0.f;
-                const float w11 = (vx1 && vy1) ? ax * mb1 : 0.f;
-                // value rows of the four corners; in-bounds rows lie in [0, S)
-                const int q00 = (int)((uint32_t)y0 * (uint32_t)Wl + (uint32_t)x0);
-                const int q10 = q00 + Wl;
-                if (vx0 && vy0) load_vec<VB>(lb + (long long)q00 * pix_bytes, r00);
-                if (vx1 && vy0) load_vec<VB>(lb + (long long)(q00 + 1) * pix_bytes, r01);
-                if (vx0 && vy1) load_vec<VB>(lb + (long long)q10 * pix_bytes, r10);
-                if (vx1 && vy1) load_vec<VB>(lb + (long long)(q10 + 1) * pix_bytes, r11);
-                float f[CPT];
-                widen<T, CPT>(r00, f);
-                axpy<CPT>(acc, w00, f);
-                widen<T, CPT>(r01, f);
-                axpy<CPT>(acc, w01, f);
-                widen<T, CPT>(r10, f);
-                axpy<CPT>(acc, w10, f);
-                widen<T, CPT>(r11, f);
-                axpy<CPT>(acc, w11, f);
+        // rolling corner pipeline over the L*K taps (level-major)
+        uint32_t v[4][NW];
+        float w[4];
+        int nl = 0, nt = 0;                  // level and index of the next tap
+        auto geometry = [&]() {
+            float u, vv;
+            load_pair<T>(locp + 2 * nt, u, vv);
+            const MsdaTap t = msda_tap(s_lvl, pix_bytes, nl, u, vv, Elem<T>::one(wp + nt));
+            ++nt;
+            if (nt == (nl + 1) * K) ++nl;
+            return t;
+        };
+        {
+            const MsdaTap t0 = geometry();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                load_vec<VB>(vb + t0.off[c], v[c]);
+                w[c] = t0.w[c];
+            }
+        }
+#pragma unroll 1
+        for (int t = 0; t < LK; ++t) {
+            const bool more = t + 1 < LK;
+            MsdaTap tn;
+            if (more) tn = geometry();
+            float f[CPT];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                widen<T, CPT>(v[c], f);
+                axpy<CPT>(acc, w[c], f);
+                if (more) load_vec<VB>(vb + tn.off[c], v[c]);
+            }
+            if (more) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) w[c] = tn.w[c];
             }
         }
 

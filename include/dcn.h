@@ -72,8 +72,10 @@ typedef enum {
  *   out    [N][Ho][Wo][C]
  *   Ho = (H + 2*pad - dil*(kh - 1) - 1) / stride + 1, Wo likewise with W, kw.
  *
- * Limits: H, W, kh, kw, stride, dil <= 65536; one image of x and of out below
- * 2^31 bytes (DCN_ERR_UNSUPPORTED otherwise).  N = 0 launches nothing and
+ * Limits: H, W, pad, stride, dil <= 65536; kh * kw <= 1024; one group's
+ * channels D * element size <= 1024 bytes (at most 32 threads per (pixel,
+ * group)); one image of x and of out below 2^31 bytes; N * Ho * Wo * G below
+ * 2^31 (DCN_ERR_UNSUPPORTED otherwise).  N = 0 launches nothing and
  * returns DCN_OK.  Offsets may be any value: a tap whose corners all fall
  * outside the map, however far, contributes 0; a NaN offset makes its tap
  * contribute 0.  Non-finite x or mask values give unspecified (but never
@@ -115,9 +117,10 @@ DCN_API int dcn_forward(const void* x, const void* offset, const void* mask, voi
  * The device contents of spatial_shapes and level_start are a precondition
  * (positive shapes, starts inside value); they are not validated, because that
  * would need a synchronisation.
- * Limits: L <= 16, K <= 64, M * D and one batch item of value and out below
- * 2^31 bytes (DCN_ERR_UNSUPPORTED otherwise).  N = 0 or Lq = 0 launches nothing
- * and returns DCN_OK.
+ * Limits: L <= 16, K <= 64, one head's channels D * element size <= 1024
+ * bytes, N * Lq * M below 2^31 (DCN_ERR_UNSUPPORTED otherwise); S below 2^31
+ * rows (a precondition, like the level table).  N = 0 or Lq = 0 launches
+ * nothing and returns DCN_OK.
  * Errors: DCN_ERR_INVALID_ARG for N < 0, Lq < 0, M, D, L or K <= 0, an unknown
  * dtype, a null pointer (N * Lq > 0) or out overlapping an input;
  * DCN_ERR_MISALIGNED when a pointer is not aligned to its element size.

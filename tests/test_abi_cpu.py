@@ -90,6 +90,7 @@ def call_dcn(lib, **kw):
     (dict(mask=MASK + 2, dtype=0), dcnb.DCN_ERR_MISALIGNED),   # f32 needs 4 bytes
     (dict(H=70000), dcnb.DCN_ERR_UNSUPPORTED),
     (dict(kh=33, kw=33, pad=16), dcnb.DCN_ERR_UNSUPPORTED),   # K > 1024
+    (dict(C=1026, G=1), dcnb.DCN_ERR_UNSUPPORTED),     # D * 2 bytes > 1024
     (dict(N=0), dcnb.DCN_OK),                          # nothing to do, nothing launched
     (dict(N=0, x=None, out=None), dcnb.DCN_OK),
 ])
@@ -117,6 +118,7 @@ def call_msda(lib, **kw):
     (dict(Lq=-1), dcnb.DCN_ERR_INVALID_ARG),
     (dict(L=17), dcnb.DCN_ERR_UNSUPPORTED),
     (dict(K=65), dcnb.DCN_ERR_UNSUPPORTED),
+    (dict(D=260), dcnb.DCN_ERR_UNSUPPORTED),           # D * 4 bytes > 1024
     (dict(shapes=None), dcnb.DCN_ERR_INVALID_ARG),
     (dict(out=MASK), dcnb.DCN_ERR_INVALID_ARG),        # out aliases loc
     (dict(out=X), dcnb.DCN_ERR_INVALID_ARG),           # out aliases value
