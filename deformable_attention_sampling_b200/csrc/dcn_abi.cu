@@ -195,8 +195,11 @@ TileShape choose_tile(int N, int Ho, int runs, int kernel_extent, int sms) {
 }
 
 template <typename T, int VB>
-const void* dcn_kernel_for(int softmax) {
+const void* dcn_kernel_for(int softmax, int kh, int kw) {
     using namespace dcnb;
+    if (kh == 3 && kw == 3)   // the common window: taps fully unrolled
+        return softmax ? (const void*)dcn_fwd_kernel<T, VB, true, 3>
+                       : (const void*)dcn_fwd_kernel<T, VB, false, 3>;
     return softmax ? (const void*)dcn_fwd_kernel<T, VB, true>
                    : (const void*)dcn_fwd_kernel<T, VB, false>;
 }
@@ -204,14 +207,14 @@ const void* dcn_kernel_for(int softmax) {
 template <typename T>
 const void* dcn_kernel_vb(int vb, int kh, int kw, int softmax) {
     switch (vb) {
-        case 32: return dcn_kernel_for<T, 32>(softmax);
-        case 16: return dcn_kernel_for<T, 16>(softmax);
-        case 8: return dcn_kernel_for<T, 8>(softmax);
-        case 4: return dcn_kernel_for<T, 4>(softmax);
+        case 32: return dcn_kernel_for<T, 32>(softmax, kh, kw);
+        case 16: return dcn_kernel_for<T, 16>(softmax, kh, kw);
+        case 8: return dcn_kernel_for<T, 8>(softmax, kh, kw);
+        case 4: return dcn_kernel_for<T, 4>(softmax, kh, kw);
         default: break;
     }
     if constexpr (sizeof(T) == 2) {
-        if (vb == 2) return dcn_kernel_for<T, 2>(softmax);
+        if (vb == 2) return dcn_kernel_for<T, 2>(softmax, kh, kw);
     }
     return nullptr;
 }
