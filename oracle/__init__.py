@@ -35,6 +35,10 @@ def bind(lib):
     lib.oracle_msda_forward.restype = ctypes.c_int
     lib.oracle_out_size.argtypes = [L] * 5
     lib.oracle_out_size.restype = L
+    lib.oracle_dcn_backward.argtypes = [dp] * 7 + [L] * 10 + [ctypes.c_int]
+    lib.oracle_dcn_backward.restype = ctypes.c_int
+    lib.oracle_msda_backward.argtypes = [dp, lp, lp, dp, dp, dp, dp, dp, dp] + [L] * 7
+    lib.oracle_msda_backward.restype = ctypes.c_int
     return lib
 
 
@@ -109,3 +113,58 @@ def msda_forward_ref(value, spatial_shapes, level_start, loc, attn):
     if rc != 0:
         raise ValueError("oracle_msda_forward rejected its arguments")
     return out
+
+
+def dcn_backward_ref(x, offset, mask, grad_out, kh, kw, stride=1, pad=1, dil=1,
+                     softmax_flag=0, groups=None):
+    """float64 gradients of dcn_forward_ref for the upstream gradient grad_out.
+
+    Returns (grad_x [N,H,W,C], grad_offset [N,Ho,Wo,G,K,2], grad_mask [N,Ho,Wo,G,K]);
+    grad_mask is with respect to the mask argument (the logits when softmax_flag = 1).
+    """
+    x = _as_f64(x)
+    offset = _as_f64(offset)
+    mask = _as_f64(mask)
+    grad_out = _as_f64(grad_out)
+    N, H, W, C = x.shape
+    G = groups if groups is not None else mask.shape[3]
+    Ho = out_size(H, kh, stride, pad, dil)
+    Wo = out_size(W, kw, stride, pad, dil)
+    K = kh * kw
+    assert offset.size == N * Ho * Wo * G * K * 2 and mask.size == N * Ho * Wo * G * K
+    assert grad_out.size == N * Ho * Wo * C, "grad_out has the wrong size"
+    gx = np.zeros_like(x)
+    goff = np.zeros((N, Ho, Wo, G, K, 2))
+    gmask = np.zeros((N, Ho, Wo, G, K))
+    rc = _load().oracle_dcn_backward(_ptr(x), _ptr(offset), _ptr(mask), _ptr(grad_out),
+                                     _ptr(gx), _ptr(goff), _ptr(gmask), N, H, W, C, G, kh, kw,
+                                     stride, pad, dil, int(softmax_flag))
+    if rc != 0:
+        raise ValueError("oracle_dcn_backward rejected its arguments")
+    return gx, goff, gmask
+
+
+def msda_backward_ref(value, spatial_shapes, level_start, loc, attn, grad_out):
+    """float64 gradients of msda_forward_ref for the upstream gradient grad_out.
+
+    Returns (grad_value [N,S,M,D], grad_loc [N,Lq,M,L,K,2], grad_attn [N,Lq,M,L,K]).
+    """
+    value = _as_f64(value)
+    loc = _as_f64(loc)
+    attn = _as_f64(attn)
+    grad_out = _as_f64(grad_out)
+    shapes = np.ascontiguousarray(np.asarray(spatial_shapes, dtype=np.int64))
+    starts = np.ascontiguousarray(np.asarray(level_start, dtype=np.int64))
+    N, S, M, D = value.shape
+    _, Lq, _, L, K = attn.shape
+    assert loc.shape == (N, Lq, M, L, K, 2) and grad_out.size == N * Lq * M * D
+    gv = np.zeros_like(value)
+    gl = np.zeros_like(loc)
+    ga = np.zeros_like(attn)
+    rc = _load().oracle_msda_backward(_ptr(value), _ptr(shapes, ctypes.c_longlong),
+                                      _ptr(starts, ctypes.c_longlong), _ptr(loc), _ptr(attn),
+                                      _ptr(grad_out), _ptr(gv), _ptr(gl), _ptr(ga), N, S, Lq,
+                                      M, D, L, K)
+    if rc != 0:
+        raise ValueError("oracle_msda_backward rejected its arguments")
+    return gv, gl, ga

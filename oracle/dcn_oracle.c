@@ -210,3 +210,199 @@ int oracle_msda_forward(const double *value, const long long *shapes,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Backward (gradients of the forward above), the plain chain rule.
+ *
+ * With L the loss and g = dL/dout, each output channel is
+ *   out = sum_k m_k * sum_corners w_corner(a_k, b_k) * v_corner,
+ * so (the bilinear weights being (1-a)(1-b), a(1-b), (1-a)b, ab with
+ * a = px - floor(px), da/dpx = 1, between integer points):
+ *   dL/dv_corner += g * m_k * w_corner                   (corner inside the map)
+ *   dL/dm_k      += g * sample_k
+ *   dL/dpx_k     += g * m_k * ((1-b)(v01 - v00) + b (v11 - v10))
+ *   dL/dpy_k     += g * m_k * ((1-a)(v10 - v00) + a (v11 - v01))
+ * with v = 0 for a corner outside the map.  At an exactly integer coordinate
+ * the floor convention (a = 0, corners x0 and x0+1) gives the right-hand
+ * derivative.  DCNv3: m = softmax(z) over K, dL/dz_k = m_k (dL/dm_k -
+ * sum_j m_j dL/dm_j).  MSDA: x = u W - 1/2, so dL/du = W dL/dx.
+ * ---------------------------------------------------------------------- */
+
+/* value of corner (xx, yy) of channel c, 0 outside the map */
+static double corner_value(const double *map, long H, long W, long pix_stride, long c,
+                           double xx, double yy)
+{
+    if (xx >= 0.0 && xx < (double)W && yy >= 0.0 && yy < (double)H)
+        return map[((long)yy * W + (long)xx) * pix_stride + c];
+    return 0.0;
+}
+
+static void corner_add(double *map, long H, long W, long pix_stride, long c, double xx,
+                       double yy, double v)
+{
+    if (xx >= 0.0 && xx < (double)W && yy >= 0.0 && yy < (double)H)
+        map[((long)yy * W + (long)xx) * pix_stride + c] += v;
+}
+
+/*
+ * DCNv3 / DCNv4 backward.  Inputs as oracle_dcn_forward plus grad_out
+ * [N][Ho][Wo][C]; outputs (overwritten) grad_x [N][H][W][C], grad_offset
+ * [N][Ho][Wo][G][K][2], grad_mask [N][Ho][Wo][G][K] (the gradient with respect
+ * to the mask argument: m itself, or the logits when softmax_flag = 1).
+ */
+int oracle_dcn_backward(const double *x, const double *offset, const double *mask,
+                        const double *grad_out, double *grad_x, double *grad_offset,
+                        double *grad_mask, long N, long H, long W, long C, long G, long kh,
+                        long kw, long stride, long pad, long dil, int softmax_flag)
+{
+    if (N < 0 || H <= 0 || W <= 0 || C <= 0 || G <= 0 || C % G != 0 || kh <= 0 ||
+        kw <= 0 || stride <= 0 || pad < 0 || dil <= 0)
+        return -1;
+    long Ho = oracle_out_size(H, kh, stride, pad, dil);
+    long Wo = oracle_out_size(W, kw, stride, pad, dil);
+    if (Ho <= 0 || Wo <= 0)
+        return -1;
+    long D = C / G;
+    long K = kh * kw;
+    double *m = (double *)malloc(sizeof(double) * (size_t)K * 2);
+    if (!m)
+        return -1;
+    double *gm = m + K;
+
+    for (long i = 0; i < N * H * W * C; ++i)
+        grad_x[i] = 0.0;
+
+    for (long n = 0; n < N; ++n)
+    for (long oy = 0; oy < Ho; ++oy)
+    for (long ox = 0; ox < Wo; ++ox)
+    for (long g = 0; g < G; ++g) {
+        long site = ((n * Ho + oy) * Wo + ox) * G + g;
+        const double *off = offset + site * K * 2;
+        const double *msk = mask + site * K;
+        double *goff = grad_offset + site * K * 2;
+        double *gmsk = grad_mask + site * K;
+        if (softmax_flag) {
+            double zmax = msk[0];
+            for (long k = 1; k < K; ++k)
+                if (msk[k] > zmax)
+                    zmax = msk[k];
+            double sum = 0.0;
+            for (long k = 0; k < K; ++k) {
+                m[k] = exp(msk[k] - zmax);
+                sum += m[k];
+            }
+            for (long k = 0; k < K; ++k)
+                m[k] = m[k] / sum;
+        } else {
+            for (long k = 0; k < K; ++k)
+                m[k] = msk[k];
+        }
+        const double *xg = x + n * H * W * C + g * D;
+        double *gxg = grad_x + n * H * W * C + g * D;
+        const double *go = grad_out + ((n * Ho + oy) * Wo + ox) * C + g * D;
+
+        for (long ix = 0; ix < kw; ++ix)
+        for (long iy = 0; iy < kh; ++iy) {
+            long k = ix * kh + iy;
+            double px = (double)(ox * stride - pad + ix * dil) + off[2 * k];
+            double py = (double)(oy * stride - pad + iy * dil) + off[2 * k + 1];
+            double x0 = floor(px), y0 = floor(py);
+            double a = px - x0, b = py - y0;
+            double gdx = 0.0, gdy = 0.0, gmk = 0.0;
+            for (long c = 0; c < D; ++c) {
+                double v00 = corner_value(xg, H, W, C, c, x0, y0);
+                double v01 = corner_value(xg, H, W, C, c, x0 + 1, y0);
+                double v10 = corner_value(xg, H, W, C, c, x0, y0 + 1);
+                double v11 = corner_value(xg, H, W, C, c, x0 + 1, y0 + 1);
+                double sample = (1 - a) * (1 - b) * v00 + a * (1 - b) * v01 +
+                                (1 - a) * b * v10 + a * b * v11;
+                gmk += go[c] * sample;
+                gdx += go[c] * m[k] * ((1 - b) * (v01 - v00) + b * (v11 - v10));
+                gdy += go[c] * m[k] * ((1 - a) * (v10 - v00) + a * (v11 - v01));
+                double gm_c = go[c] * m[k];
+                corner_add(gxg, H, W, C, c, x0, y0, gm_c * (1 - a) * (1 - b));
+                corner_add(gxg, H, W, C, c, x0 + 1, y0, gm_c * a * (1 - b));
+                corner_add(gxg, H, W, C, c, x0, y0 + 1, gm_c * (1 - a) * b);
+                corner_add(gxg, H, W, C, c, x0 + 1, y0 + 1, gm_c * a * b);
+            }
+            goff[2 * k] = gdx;
+            goff[2 * k + 1] = gdy;
+            gm[k] = gmk;
+        }
+        if (softmax_flag) {
+            double dot = 0.0;
+            for (long k = 0; k < K; ++k)
+                dot += m[k] * gm[k];
+            for (long k = 0; k < K; ++k)
+                gmsk[k] = m[k] * (gm[k] - dot);
+        } else {
+            for (long k = 0; k < K; ++k)
+                gmsk[k] = gm[k];
+        }
+    }
+    free(m);
+    return 0;
+}
+
+/*
+ * MSDeformAttn core backward.  Inputs as oracle_msda_forward plus grad_out
+ * [N][Lq][M*D]; outputs (overwritten) grad_value [N][S][M][D], grad_loc
+ * [N][Lq][M][L][K][2], grad_attn [N][Lq][M][L][K].
+ */
+int oracle_msda_backward(const double *value, const long long *shapes,
+                         const long long *level_start, const double *loc,
+                         const double *attn, const double *grad_out, double *grad_value,
+                         double *grad_loc, double *grad_attn, long N, long S, long Lq, long M,
+                         long D, long L, long K)
+{
+    if (N < 0 || S <= 0 || Lq < 0 || M <= 0 || D <= 0 || L <= 0 || K <= 0)
+        return -1;
+    for (long l = 0; l < L; ++l) {
+        if (shapes[2 * l] <= 0 || shapes[2 * l + 1] <= 0 || level_start[l] < 0 ||
+            level_start[l] + shapes[2 * l] * shapes[2 * l + 1] > S)
+            return -1;
+    }
+    for (long i = 0; i < N * S * M * D; ++i)
+        grad_value[i] = 0.0;
+    for (long i = 0; i < N * Lq * M * L * K; ++i) {
+        grad_attn[i] = 0.0;
+        grad_loc[2 * i] = 0.0;
+        grad_loc[2 * i + 1] = 0.0;
+    }
+    for (long n = 0; n < N; ++n)
+    for (long q = 0; q < Lq; ++q)
+    for (long h = 0; h < M; ++h)
+    for (long c = 0; c < D; ++c) {
+        double go = grad_out[(n * Lq + q) * M * D + h * D + c];
+        for (long l = 0; l < L; ++l) {
+            long Hl = (long)shapes[2 * l];
+            long Wl = (long)shapes[2 * l + 1];
+            long off = ((n * S + (long)level_start[l]) * M + h) * D;
+            const double *lvl = value + off;
+            double *glvl = grad_value + off;
+            for (long k = 0; k < K; ++k) {
+                long t = (((n * Lq + q) * M + h) * L + l) * K + k;
+                double A = attn[t];
+                double x = loc[2 * t] * (double)Wl - 0.5;
+                double y = loc[2 * t + 1] * (double)Hl - 0.5;
+                double x0 = floor(x), y0 = floor(y);
+                double a = x - x0, b = y - y0;
+                double v00 = corner_value(lvl, Hl, Wl, M * D, c, x0, y0);
+                double v01 = corner_value(lvl, Hl, Wl, M * D, c, x0 + 1, y0);
+                double v10 = corner_value(lvl, Hl, Wl, M * D, c, x0, y0 + 1);
+                double v11 = corner_value(lvl, Hl, Wl, M * D, c, x0 + 1, y0 + 1);
+                double sample = (1 - a) * (1 - b) * v00 + a * (1 - b) * v01 +
+                                (1 - a) * b * v10 + a * b * v11;
+                grad_attn[t] += go * sample;
+                grad_loc[2 * t] += go * A * ((1 - b) * (v01 - v00) + b * (v11 - v10)) * Wl;
+                grad_loc[2 * t + 1] += go * A * ((1 - a) * (v10 - v00) + a * (v11 - v01)) * Hl;
+                double ga = go * A;
+                corner_add(glvl, Hl, Wl, M * D, c, x0, y0, ga * (1 - a) * (1 - b));
+                corner_add(glvl, Hl, Wl, M * D, c, x0 + 1, y0, ga * a * (1 - b));
+                corner_add(glvl, Hl, Wl, M * D, c, x0, y0 + 1, ga * (1 - a) * b);
+                corner_add(glvl, Hl, Wl, M * D, c, x0 + 1, y0 + 1, ga * a * b);
+            }
+        }
+    }
+    return 0;
+}

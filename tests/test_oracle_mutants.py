@@ -4,6 +4,8 @@ Each mutant is a copy of the C oracle with one planted mistake: a dropped
 term, a wrong sign, index or bound, a transposed operand.  It is compiled into
 a temporary library, swapped in for the real one, and the pin battery of
 test_oracle_pins is run against it: every mutant must fail at least one pin.
+Mistakes planted in the backward functions face the battery of
+test_oracle_backward_pins (adjoint identity, finite differences).
 The real oracle source is never modified.
 """
 import ctypes
@@ -14,6 +16,7 @@ import pytest
 
 import oracle
 from oracle import build as oracle_build
+from tests import test_oracle_backward_pins as bwd
 from tests import test_oracle_pins as pins
 from tests.conftest import read_golden
 
@@ -41,6 +44,31 @@ MUTANTS = {
     "msda head stride": ("+ h) * D;", ") * D;"),
 }
 
+# mistakes planted in the backward functions, caught by the backward pins
+MUTANTS_BWD = {
+    "dcn d/dx drops (1-b)": ("gdx += go[c] * m[k] * ((1 - b) * (v01 - v00)",
+                             "gdx += go[c] * m[k] * ((v01 - v00)"),
+    "dcn d/dy uses the x difference": ("gdy += go[c] * m[k] * ((1 - a) * (v10 - v00)",
+                                       "gdy += go[c] * m[k] * ((1 - a) * (v01 - v00)"),
+    "dcn grad_x corner swapped": ("corner_add(gxg, H, W, C, c, x0 + 1, y0, gm_c * a * (1 - b));",
+                                  "corner_add(gxg, H, W, C, c, x0, y0 + 1, gm_c * a * (1 - b));"),
+    "dcn grad_x misses m": ("double gm_c = go[c] * m[k];", "double gm_c = go[c];"),
+    "dcn softmax jacobian sign": ("gmsk[k] = m[k] * (gm[k] - dot);", "gmsk[k] = m[k] * (gm[k] + dot);"),
+    "dcn grad_mask of the sample": ("gmk += go[c] * sample;", "gmk += go[c] * v00;"),
+    "msda grad_loc misses W": ("* ((1 - b) * (v01 - v00) + b * (v11 - v10)) * Wl;",
+                               "* ((1 - b) * (v01 - v00) + b * (v11 - v10));"),
+    "msda grad_value misses A": ("double ga = go * A;", "double ga = go;"),
+    "msda grad_attn": ("grad_attn[t] += go * sample;", "grad_attn[t] += sample;"),
+}
+
+PIN_TESTS_BWD = [
+    (bwd.test_dcn_grad_x_is_the_adjoint, [dict(case=c) for c in bwd.DCN_CASES[:2]]),
+    (bwd.test_dcn_offset_and_mask_gradients_match_finite_differences,
+     [dict(case=c) for c in bwd.DCN_CASES[:2]]),
+    (bwd.test_msda_grad_value_is_the_adjoint, [{}]),
+    (bwd.test_msda_loc_and_attn_gradients_match_finite_differences, [{}]),
+]
+
 PIN_TESTS = [
     (pins.test_bilinear_worked_example, [{}]),
     (pins.test_spike_1d, [{}]),
@@ -64,9 +92,9 @@ PIN_TESTS = [
 ]
 
 
-def _failures():
+def _failures(battery=PIN_TESTS):
     failed = []
-    for fn, param_sets in PIN_TESTS:
+    for fn, param_sets in battery:
         for params in param_sets:
             kwargs = dict(params)
             if "golden" in inspect.signature(fn).parameters:
@@ -80,6 +108,23 @@ def _failures():
 
 def test_real_oracle_passes_the_battery():
     assert _failures() == []
+    assert _failures(PIN_TESTS_BWD) == []
+
+
+def _install_mutant(original, planted, tmp_path, monkeypatch):
+    src = open(oracle_build.SRC).read()
+    assert src.count(original) >= 1, f"mutation site not found: {original}"
+    mutant_src = tmp_path / "mutant.c"
+    mutant_src.write_text(src.replace(original, planted, 1))
+    lib_path = oracle_build.compile_oracle(str(mutant_src), str(tmp_path / "libmutant.so"),
+                                           extra_flags=("-Wno-error",))
+    monkeypatch.setattr(oracle, "_lib", oracle.bind(ctypes.CDLL(lib_path)))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS_BWD))
+def test_backward_mutant_is_caught(name, tmp_path, monkeypatch):
+    _install_mutant(*MUTANTS_BWD[name], tmp_path, monkeypatch)
+    assert _failures(PIN_TESTS_BWD), f"no backward pin caught the mutant '{name}'"
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
