@@ -1,10 +1,12 @@
 """Benchmark of the deformable sampling-aggregation forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--pass forward|backward]
 
 One step is one dcn_forward (or msda_forward) call over one full batch of the
 workload; the default workload is DCNv4 fp16, N=64, 56x56, C=64, G=4, 3x3.
+`--pass backward` times dcn_backward (msda_backward) instead: one call = the
+zero fill of the float32 accumulator, the gradient kernel and the rounding.
 Prints ONE JSON line on stdout (rank 0); diagnostics go to stderr.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
@@ -218,6 +220,14 @@ class DcnRunner:
         return [(s["x"], self.host["x"]), (s["offset"], self.host["offset"]),
                 (s["mask"], self.host["mask"])]
 
+    def outputs_of(self, s):
+        return [s["out"]]
+
+    kernel = "dcn_fwd_kernel"
+
+    def bytes_per_step(self):
+        return self.w.compulsory_bytes()
+
 
 class MsdaRunner:
     def __init__(self, w, seed, device):
@@ -251,17 +261,127 @@ class MsdaRunner:
         return [(s[k], self.host[k]) for k in ("value", "spatial_shapes", "level_start", "loc",
                                                "attn")]
 
+    def outputs_of(self, s):
+        return [s["out"]]
 
-def make_runner(w, seed, device):
-    return (DcnRunner if isinstance(w, gen.DcnWorkload) else MsdaRunner)(w, seed, device)
+    kernel = "msda_fwd_kernel"
+
+    def bytes_per_step(self):
+        return self.w.compulsory_bytes()
+
+
+class DcnBwdRunner(DcnRunner):
+    """One step = one dcn_backward call: zero fill of the float32 grad_x
+    accumulator, the gradient kernel, rounding into grad_x (16-bit data)."""
+    kernel = "dcn_bwd_kernel (+ zero fill, rounding)"
+
+    def __init__(self, w, seed, device):
+        super().__init__(w, seed, device)
+        self.host["grad_out"] = gen.grad_out((w.N, w.Ho, w.Wo, w.C), w.dtype, seed)
+        self.ws_bytes = self.dcnb.dcn_backward_workspace_size(w.N, w.H, w.W, w.C, self.code)
+
+    def alloc_set(self):
+        d = {k: v.to(self.device) for k, v in self.host.items()}
+        d["grad_x"] = torch.empty_like(d["x"])
+        d["grad_offset"] = torch.empty_like(d["offset"])
+        d["grad_mask"] = torch.empty_like(d["mask"])
+        d["ws"] = (torch.empty(self.ws_bytes // 4, dtype=torch.float32, device=self.device)
+                   if self.ws_bytes > 0 else None)
+        return d
+
+    def launcher(self, s, stream):
+        w, lib = self.w, self.lib
+        ws = s["ws"].data_ptr() if s["ws"] is not None else None
+        args = (s["x"].data_ptr(), s["offset"].data_ptr(), s["mask"].data_ptr(),
+                s["grad_out"].data_ptr(), s["grad_x"].data_ptr(), s["grad_offset"].data_ptr(),
+                s["grad_mask"].data_ptr(), ws, self.ws_bytes, w.N, w.H, w.W, w.C, w.G, w.kh,
+                w.kw, w.stride, w.pad, w.dil, w.softmax_flag, self.code, stream)
+
+        def go():
+            st = lib.dcn_backward(*args)
+            if st != 0:
+                raise self.dcnb.DcnError(st, "dcn_backward")
+        return go
+
+    def inputs_of(self, s):
+        return super().inputs_of(s) + [(s["grad_out"], self.host["grad_out"])]
+
+    def outputs_of(self, s):
+        return [s["grad_x"], s["grad_offset"], s["grad_mask"]]
+
+    def bytes_per_step(self):
+        return self.w.backward_bytes()
+
+
+class MsdaBwdRunner(MsdaRunner):
+    """One step = one msda_backward call (zero fill, gradient kernel, and the
+    rounding pass for 16-bit data)."""
+    kernel = "msda_bwd_kernel (+ zero fill, rounding)"
+
+    def __init__(self, w, seed, device):
+        super().__init__(w, seed, device)
+        self.host["grad_out"] = gen.grad_out((w.N, w.queries, w.M * w.D), w.dtype, seed)
+        self.ws_bytes = self.dcnb.msda_backward_workspace_size(w.N, w.S, w.M, w.D, self.code)
+
+    def alloc_set(self):
+        d = {k: v.to(self.device) for k, v in self.host.items()}
+        d["grad_value"] = torch.empty_like(d["value"])
+        d["grad_loc"] = torch.empty_like(d["loc"])
+        d["grad_attn"] = torch.empty_like(d["attn"])
+        d["ws"] = (torch.empty(self.ws_bytes // 4, dtype=torch.float32, device=self.device)
+                   if self.ws_bytes > 0 else None)
+        return d
+
+    def launcher(self, s, stream):
+        w, lib = self.w, self.lib
+        ws = s["ws"].data_ptr() if s["ws"] is not None else None
+        args = (s["value"].data_ptr(), s["spatial_shapes"].data_ptr(),
+                s["level_start"].data_ptr(), s["loc"].data_ptr(), s["attn"].data_ptr(),
+                s["grad_out"].data_ptr(), s["grad_value"].data_ptr(), s["grad_loc"].data_ptr(),
+                s["grad_attn"].data_ptr(), ws, self.ws_bytes, w.N, w.S, w.queries, w.M, w.D,
+                w.L, w.K, self.code, stream)
+
+        def go():
+            st = lib.msda_backward(*args)
+            if st != 0:
+                raise self.dcnb.DcnError(st, "msda_backward")
+        return go
+
+    def inputs_of(self, s):
+        return super().inputs_of(s) + [(s["grad_out"], self.host["grad_out"])]
+
+    def outputs_of(self, s):
+        return [s["grad_value"], s["grad_loc"], s["grad_attn"]]
+
+    def bytes_per_step(self):
+        return self.w.backward_bytes()
+
+
+def make_runner(w, seed, device, backward=False):
+    dcn = isinstance(w, gen.DcnWorkload)
+    if backward:
+        return (DcnBwdRunner if dcn else MsdaBwdRunner)(w, seed, device)
+    return (DcnRunner if dcn else MsdaRunner)(w, seed, device)
 
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_step(w, seed):
+def oracle_step(w, seed, backward=False):
     """Run the float64 oracle once on workload w; returns (seconds, taps)."""
     import oracle
-    if isinstance(w, gen.DcnWorkload):
+    if backward and isinstance(w, gen.DcnWorkload):
+        inp = gen.dcn_inputs(w, seed=seed)
+        go = gen.grad_out((w.N, w.Ho, w.Wo, w.C), w.dtype, seed)
+        t = time.perf_counter()
+        oracle.dcn_backward_ref(inp["x"], inp["offset"], inp["mask"], go, w.kh, w.kw, w.stride,
+                                w.pad, w.dil, w.softmax_flag)
+    elif backward:
+        inp = gen.msda_inputs(w, seed=seed)
+        go = gen.grad_out((w.N, w.queries, w.M * w.D), w.dtype, seed)
+        t = time.perf_counter()
+        oracle.msda_backward_ref(inp["value"], inp["spatial_shapes"], inp["level_start"],
+                                 inp["loc"], inp["attn"], go)
+    elif isinstance(w, gen.DcnWorkload):
         inp = gen.dcn_inputs(w, seed=seed)
         t = time.perf_counter()
         oracle.dcn_forward_ref(inp["x"], inp["offset"], inp["mask"], w.kh, w.kw, w.stride,
@@ -282,19 +402,20 @@ def sample_of(w, n_images):
     return gen.scaled(w, N=1, Lq=max(1, min(w.queries, n_images * 64)))
 
 
-def cpu_baseline(w, budget_s=10.0):
+def cpu_baseline(w, budget_s=10.0, backward=False):
     """The oracle as it stands, single-threaded, on a bounded sample of the
     workload, repeated until about `budget_s` seconds of CPU work."""
     s = sample_of(w, 8)
     total_t, total_taps, reps = 0.0, 0, 0
     while total_t < budget_s or reps == 0:
-        dt, taps = oracle_step(s, seed=reps)
+        dt, taps = oracle_step(s, seed=reps, backward=backward)
         total_t += dt
         total_taps += taps
         reps += 1
     desc = (f"{reps} x oracle on {s.name} with N={s.N}" +
             (f", Lq={s.queries}" if isinstance(s, gen.MsdaWorkload) else "") +
-            f" ({s.taps()} taps each), single thread, float64")
+            f" ({s.taps()} taps each), single thread, float64" +
+            (", backward" if backward else ""))
     return {"value": total_taps / total_t, "unit": "taps/s", "cores": 1, "kind": "oracle",
             "sample": desc, "host_cpus": os.cpu_count()}
 
@@ -338,8 +459,9 @@ def run_b200(args):
         raise RuntimeError("libdcn_b200.so is not built (python -m "
                            "deformable_attention_sampling_b200.build)")
 
-    runner = make_runner(w, seed=1000 + rank, device=device)
-    bytes_per_step = w.compulsory_bytes()
+    backward = args.pass_ == "backward"
+    runner = make_runner(w, seed=1000 + rank, device=device, backward=backward)
+    bytes_per_step = runner.bytes_per_step()
     l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
     n_sets = max(2, int(np.ceil(3 * l2_bytes / bytes_per_step)))
     sets = [runner.alloc_set() for _ in range(n_sets)]
@@ -374,15 +496,17 @@ def run_b200(args):
     # end to end through the public call with host buffers: H2D of the step's
     # inputs from pinned memory, the call, D2H of the output, every step
     e2e_steps = min(args.steps, 200)
-    pinned_out = torch.empty(sets[0]["out"].shape, dtype=sets[0]["out"].dtype).pin_memory()
+    pinned_out = [(torch.empty(o.shape, dtype=o.dtype).pin_memory(), o)
+                  for o in runner.outputs_of(sets[0])]
     pinned_in = [(dev, host.pin_memory()) for dev, host in runner.inputs_of(sets[0])]
     h2d = sum(h.numel() * h.element_size() for _, h in pinned_in)
-    d2h = pinned_out.numel() * pinned_out.element_size()
+    d2h = sum(h.numel() * h.element_size() for h, _ in pinned_out)
     for _ in range(2):
         for dev, host in pinned_in:
             dev.copy_(host, non_blocking=True)
         launch[0]()
-        pinned_out.copy_(sets[0]["out"], non_blocking=True)
+        for host, dev in pinned_out:
+            host.copy_(dev, non_blocking=True)
     barrier(world, device)
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
@@ -391,7 +515,8 @@ def run_b200(args):
         for dev, host in pinned_in:
             dev.copy_(host, non_blocking=True)
         launch[0]()
-        pinned_out.copy_(sets[0]["out"], non_blocking=True)
+        for host, dev in pinned_out:
+            host.copy_(dev, non_blocking=True)
     e_end.record(stream)
     e_end.synchronize()
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world, device) / e2e_steps
@@ -403,12 +528,12 @@ def run_b200(args):
     achieved = bytes_per_step / (ms_local / args.steps * 1e-3) / 1e9
     traffic = None
     if (NCU_TRAFFIC["source_sha256"] == kernel_source_hash()
-            and w.name == gen.HEADLINE):
+            and w.name == gen.HEADLINE and not backward):
         traffic = NCU_TRAFFIC["bytes_per_launch"]
 
     result = None
     if rank == 0:
-        kernel = "dcn_fwd_kernel" if isinstance(w, gen.DcnWorkload) else "msda_fwd_kernel"
+        kernel = runner.kernel
         config = {"workload": w.name, "global_batch": w.N * world,
                   "per_gpu_batch": w.N, "dtype_storage": w.dtype, "accumulate": "f32",
                   "l2": f"{n_sets} rotating input/output sets ({n_sets * bytes_per_step / 1e6:.0f} MB"
@@ -422,7 +547,7 @@ def run_b200(args):
             config.update({"M": w.M, "D": w.D, "levels": [list(s) for s in w.shapes],
                            "K": w.K, "Lq": w.queries})
         result = {
-            "metric": METRIC if w.name == gen.HEADLINE else f"sampled taps/s ({w.name})",
+            "metric": metric_name(w, backward),
             "value": value,
             "unit": "taps/s",
             "n_gpus": world,
@@ -450,7 +575,13 @@ def run_b200(args):
             "clocks": sampler.summary(),
         }
         if world == 1:
-            result["cpu_baseline"] = cpu_baseline(w)
+            result["cpu_baseline"] = cpu_baseline(w, backward=backward)
+        if backward:
+            result["pass"] = "backward"
+            result["roofline"]["note"] = (
+                "timed over the whole dcn_backward / msda_backward call (zero fill, gradient "
+                "kernel, rounding); algorithmic bytes = inputs + grad_out read, three "
+                "gradients written once, no float32 accumulator traffic")
     if world > 1:
         import torch.distributed as dist
         dist.barrier(device_ids=[device.index])
@@ -466,8 +597,9 @@ def run_reference(args):
         return None
     w = gen.WORKLOADS[args.workload]
     # size one step so that warm-up plus timed steps take about a minute
+    backward = args.pass_ == "backward"
     probe = sample_of(w, 1)
-    dt, taps = oracle_step(probe, seed=0)
+    dt, taps = oracle_step(probe, seed=0, backward=backward)
     rate = taps / dt
     budget = 60.0 / max(1, args.steps + args.warmup)
     if isinstance(w, gen.DcnWorkload):
@@ -483,10 +615,10 @@ def run_reference(args):
         q = max(1, min(w.queries, int(budget * rate / per_query)))
         step_w = gen.scaled(w, N=1, Lq=q)
     for i in range(args.warmup):
-        oracle_step(step_w, seed=i)
+        oracle_step(step_w, seed=i, backward=backward)
     total_t, total_taps = 0.0, 0
     for i in range(args.steps):
-        t, taps = oracle_step(step_w, seed=args.warmup + i)
+        t, taps = oracle_step(step_w, seed=args.warmup + i, backward=backward)
         total_t += t
         total_taps += taps
     value = total_taps / total_t
@@ -496,7 +628,7 @@ def run_reference(args):
               + f" ({step_w.taps()} taps), single thread, float64")
     return {
         "impl": "reference",
-        "metric": METRIC if w.name == gen.HEADLINE else f"sampled taps/s ({w.name})",
+        "metric": metric_name(w, backward),
         "value": value,
         "unit": "taps/s",
         "n_gpus": world,
@@ -516,6 +648,12 @@ def run_reference(args):
     }
 
 
+def metric_name(w, backward):
+    if backward:
+        return f"backward sampled taps/s ({w.name})"
+    return METRIC if w.name == gen.HEADLINE else f"sampled taps/s ({w.name})"
+
+
 def main():
     p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     p.add_argument("--gpus", type=int, default=1)
@@ -523,6 +661,8 @@ def main():
     p.add_argument("--warmup", type=int, default=200)
     p.add_argument("--impl", default="b200", choices=["b200", "reference"])
     p.add_argument("--workload", default=gen.HEADLINE, choices=sorted(gen.WORKLOADS))
+    p.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
+                   help="time the forward call (default) or the backward call")
     args = p.parse_args()
     if args.warmup < 3:
         p.error("--warmup must be at least 3")

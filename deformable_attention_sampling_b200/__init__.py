@@ -1,13 +1,15 @@
 """Deformable sampling-aggregation on NVIDIA B200 (sm_100a).
 
 DCNv3 / DCNv4 deformable convolution core and the multi-scale deformable
-attention (MSDeformAttn) core, forward, as hand-written CUDA kernels behind a
+attention (MSDeformAttn) core, forward and backward, as hand-written CUDA kernels behind a
 C interface (include/dcn.h, libdcn_b200.so).  This package is the thin Python
 binding: it marshals pointers, sizes and streams and runs nothing itself.
 
     import deformable_attention_sampling_b200 as dcnb
     out = dcnb.dcn(x, offset, mask)          # torch CUDA tensors, NHWC
     out = dcnb.msda(value, shapes, starts, loc, attn)
+    gx, goff, gmask = dcnb.dcn_grad(x, offset, mask, grad_out)
+    gv, gloc, gattn = dcnb.msda_grad(value, shapes, starts, loc, attn, grad_out)
 """
 from ._binding import (  # noqa: F401
     DCN_ERR_CUDA,
@@ -20,7 +22,10 @@ from ._binding import (  # noqa: F401
     SIGNATURES,
     DcnError,
     dcn,
+    dcn_backward,
+    dcn_backward_workspace_size,
     dcn_forward,
+    dcn_grad,
     dcn_last_cuda_error,
     dcn_launch_count,
     dcn_output_size,
@@ -29,5 +34,8 @@ from ._binding import (  # noqa: F401
     dtype_code,
     library,
     msda,
+    msda_backward,
+    msda_backward_workspace_size,
     msda_forward,
+    msda_grad,
 )

@@ -25,9 +25,14 @@ DTYPE_CODES = {"f32": 0, "f16": 1, "bf16": 2}
 # every symbol include/dcn.h declares, with its ctypes signature
 _VP = ctypes.c_void_p
 _I = ctypes.c_int
+_LL = ctypes.c_longlong
 SIGNATURES = {
     "dcn_forward": (_I, [_VP, _VP, _VP, _VP] + [_I] * 12 + [_VP]),
     "msda_forward": (_I, [_VP] * 6 + [_I] * 7 + [_VP]),
+    "dcn_backward_workspace_size": (_LL, [_I] * 5),
+    "dcn_backward": (_I, [_VP] * 8 + [_LL] + [_I] * 12 + [_VP]),
+    "msda_backward_workspace_size": (_LL, [_I] * 5),
+    "msda_backward": (_I, [_VP] * 10 + [_LL] + [_I] * 8 + [_VP]),
     "dcn_output_size": (_I, [_I] * 5),
     "dcn_status_string": (ctypes.c_char_p, [_I]),
     "dcn_last_cuda_error": (_I, []),
@@ -108,6 +113,37 @@ def msda_forward(value, spatial_shapes, level_start, sampling_loc, attn_w, out, 
                                 _ptr(sampling_loc), _ptr(attn_w), _ptr(out), N, Lq, M, D, L,
                                 K, dtype, _stream(stream)),
            "msda_forward")
+
+
+def dcn_backward_workspace_size(N, H, W, C, dtype):
+    return int(_load().dcn_backward_workspace_size(N, H, W, C, dtype))
+
+
+def dcn_backward(x, offset, mask, grad_out, grad_x, grad_offset, grad_mask, workspace,
+                 workspace_bytes, N, H, W, C, G, kh, kw, stride, pad, dil, softmax_flag, dtype,
+                 stream=None):
+    """C dcn_backward; raises DcnError on a non-OK status."""
+    _check(_load().dcn_backward(_ptr(x), _ptr(offset), _ptr(mask), _ptr(grad_out), _ptr(grad_x),
+                                _ptr(grad_offset), _ptr(grad_mask), _ptr(workspace),
+                                workspace_bytes, N, H, W, C, G, kh, kw, stride, pad, dil,
+                                softmax_flag, dtype, _stream(stream)),
+           "dcn_backward")
+
+
+def msda_backward_workspace_size(N, S, M, D, dtype):
+    return int(_load().msda_backward_workspace_size(N, S, M, D, dtype))
+
+
+def msda_backward(value, spatial_shapes, level_start, sampling_loc, attn_w, grad_out,
+                  grad_value, grad_loc, grad_attn, workspace, workspace_bytes, N, S, Lq, M, D,
+                  L, K, dtype, stream=None):
+    """C msda_backward; raises DcnError on a non-OK status."""
+    _check(_load().msda_backward(_ptr(value), _ptr(spatial_shapes), _ptr(level_start),
+                                 _ptr(sampling_loc), _ptr(attn_w), _ptr(grad_out),
+                                 _ptr(grad_value), _ptr(grad_loc), _ptr(grad_attn),
+                                 _ptr(workspace), workspace_bytes, N, S, Lq, M, D, L, K, dtype,
+                                 _stream(stream)),
+           "msda_backward")
 
 
 def dcn_output_size(n_in, k, stride, pad, dil):
@@ -203,3 +239,74 @@ def msda(value, spatial_shapes, level_start, sampling_loc, attn_w, out=None, str
     msda_forward(value, spatial_shapes, level_start, sampling_loc, attn_w, out, N, Lq, M, D, L,
                  K, dtype_code(value), stream)
     return out
+
+
+def _workspace(nbytes, device, workspace):
+    """A caller-given workspace tensor, or a new one of nbytes (16-byte aligned)."""
+    import torch
+    if nbytes <= 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(nbytes // 4, dtype=torch.float32, device=device)
+    _require(workspace.is_cuda and workspace.is_contiguous(), "workspace must be a CUDA tensor")
+    have = workspace.numel() * workspace.element_size()
+    _require(have >= nbytes, f"workspace holds {have} bytes, {nbytes} needed")
+    return workspace, have
+
+
+def dcn_grad(x, offset, mask, grad_out, kh=3, kw=3, stride=1, pad=1, dil=1, softmax_flag=0,
+             workspace=None, stream=None):
+    """dcn_backward on torch CUDA tensors: returns (grad_x, grad_offset, grad_mask).
+
+    The float32 accumulator for grad_x of 16-bit data comes from `workspace`
+    when given (a CUDA tensor of at least dcn_backward_workspace_size bytes),
+    else a new tensor.
+    """
+    import torch
+    _require(x.dim() == 4 and mask.dim() == 5 and offset.dim() == 6,
+             "expected x [N,H,W,C], offset [N,Ho,Wo,G,K,2], mask [N,Ho,Wo,G,K]")
+    N, H, W, C = x.shape
+    G = mask.shape[3]
+    Ho = dcn_output_size(H, kh, stride, pad, dil)
+    Wo = dcn_output_size(W, kw, stride, pad, dil)
+    K = kh * kw
+    _require(tuple(offset.shape) == (N, Ho, Wo, G, K, 2), "offset has the wrong shape")
+    _require(tuple(mask.shape) == (N, Ho, Wo, G, K), "mask has the wrong shape")
+    _require(tuple(grad_out.shape) == (N, Ho, Wo, C), "grad_out has the wrong shape")
+    for t in (offset, mask, grad_out):
+        _require(t.dtype == x.dtype, "mixed dtypes")
+    for t in (x, offset, mask, grad_out):
+        _require(t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors")
+    code = dtype_code(x)
+    ws, ws_bytes = _workspace(dcn_backward_workspace_size(N, H, W, C, code), x.device, workspace)
+    gx = torch.empty_like(x)
+    goff = torch.empty_like(offset)
+    gmask = torch.empty_like(mask)
+    dcn_backward(x, offset, mask, grad_out, gx, goff, gmask, ws, ws_bytes, N, H, W, C, G, kh,
+                 kw, stride, pad, dil, softmax_flag, code, stream)
+    return gx, goff, gmask
+
+
+def msda_grad(value, spatial_shapes, level_start, sampling_loc, attn_w, grad_out,
+              workspace=None, stream=None):
+    """msda_backward on torch CUDA tensors: returns (grad_value, grad_loc, grad_attn)."""
+    import torch
+    N, S, M, D = value.shape
+    _, Lq, _, L, K = attn_w.shape
+    _require(tuple(sampling_loc.shape) == (N, Lq, M, L, K, 2), "sampling_loc has the wrong shape")
+    _require(tuple(grad_out.shape) == (N, Lq, M * D), "grad_out has the wrong shape")
+    _require(spatial_shapes.dtype == torch.int64 and level_start.dtype == torch.int64,
+             "spatial_shapes / level_start must be int64")
+    for t in (sampling_loc, attn_w, grad_out):
+        _require(t.dtype == value.dtype, "mixed dtypes")
+    for t in (value, spatial_shapes, level_start, sampling_loc, attn_w, grad_out):
+        _require(t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors")
+    code = dtype_code(value)
+    ws, ws_bytes = _workspace(msda_backward_workspace_size(N, S, M, D, code), value.device,
+                              workspace)
+    gv = torch.empty_like(value)
+    gl = torch.empty_like(sampling_loc)
+    ga = torch.empty_like(attn_w)
+    msda_backward(value, spatial_shapes, level_start, sampling_loc, attn_w, grad_out, gv, gl, ga,
+                  ws, ws_bytes, N, S, Lq, M, D, L, K, code, stream)
+    return gv, gl, ga

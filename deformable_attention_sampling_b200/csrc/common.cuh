@@ -83,7 +83,8 @@ __device__ __forceinline__ void store_vec<2>(void* p, const uint32_t* w) {
 // ------------------------------------------------------ element widening --
 
 // Element traits: exact widening of stored words to float32 and rounding of
-// float32 results back to the storage type (round to nearest even).
+// float32 results back to the storage type (round to nearest even; `from`
+// rounds one value).
 template <typename T>
 struct Elem;
 
@@ -95,6 +96,7 @@ struct Elem<float> {
     static __device__ __forceinline__ float one(const float* p) { return *p; }
     static __device__ __forceinline__ uint32_t pack2(float a, float) { return __float_as_uint(a); }
     static __device__ __forceinline__ uint32_t pack1(float a) { return __float_as_uint(a); }
+    static __device__ __forceinline__ float from(float a) { return a; }
 };
 
 template <>
@@ -114,6 +116,7 @@ struct Elem<__half> {
     static __device__ __forceinline__ uint32_t pack1(float a) {
         return (uint32_t)__half_as_ushort(__float2half_rn(a));
     }
+    static __device__ __forceinline__ __half from(float a) { return __float2half_rn(a); }
 };
 
 template <>
@@ -133,6 +136,9 @@ struct Elem<__nv_bfloat16> {
     }
     static __device__ __forceinline__ uint32_t pack1(float a) {
         return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a));
+    }
+    static __device__ __forceinline__ __nv_bfloat16 from(float a) {
+        return __float2bfloat16_rn(a);
     }
 };
 

@@ -76,6 +76,15 @@ class DcnWorkload:
         out = self.pixels() * self.C
         return (x + om + out) * es
 
+    def backward_bytes(self):
+        """x, offsets, masks and grad_out read once; grad_x, grad_offset and
+        grad_mask written once (no accumulator traffic)."""
+        es = DTYPES[self.dtype].itemsize
+        x = self.N * self.H * self.W * self.C
+        om = self.pixels() * self.G * self.K * 3
+        out = self.pixels() * self.C
+        return (2 * x + 2 * om + out) * es
+
 
 @dataclass(frozen=True)
 class MsdaWorkload:
@@ -114,6 +123,15 @@ class MsdaWorkload:
         w = self.taps()
         out = self.N * self.queries * self.M * self.D
         return (value + loc + w + out) * es
+
+    def backward_bytes(self):
+        """value, locations, weights and grad_out read once; grad_value,
+        grad_loc and grad_attn written once (no accumulator traffic)."""
+        es = DTYPES[self.dtype].itemsize
+        value = self.N * self.S * self.M * self.D
+        lw = self.taps() * 3
+        out = self.N * self.queries * self.M * self.D
+        return (2 * value + 2 * lw + out) * es
 
 
 WORKLOADS = {w.name: w for w in [
@@ -185,6 +203,14 @@ def msda_inputs(w, seed=0):
         "attn": _round(attn, w.dtype),
         "logits": logits,
     }
+
+
+def grad_out(shape, dtype, seed=0):
+    """Upstream gradient for a backward pass: N(0, 1) of the output's shape,
+    rounded to the dtype (a CPU tensor).  Drawn from its own stream, so the
+    forward inputs of the same seed are unchanged."""
+    rng = np.random.default_rng([seed, 0x6772])
+    return _round(rng.normal(0.0, 1.0, size=tuple(shape)), dtype)
 
 
 def scaled(w, **changes):

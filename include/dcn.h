@@ -1,7 +1,7 @@
 /*
  * dcn.h - C interface of libdcn_b200.so: deformable sampling-aggregation
  * (DCNv3 / DCNv4 core) and multi-scale deformable attention (MSDeformAttn core)
- * forward on NVIDIA B200 (sm_100a).
+ * forward and backward on NVIDIA B200 (sm_100a).
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
@@ -129,6 +129,101 @@ DCN_API int msda_forward(const void* value, const int64_t* spatial_shapes,
                  const int64_t* level_start, const void* sampling_loc,
                  const void* attn_w, void* out, int N, int Lq, int M, int D,
                  int L, int K, int dtype, void* stream);
+
+/*
+ * dcn_backward_workspace_size - bytes of scratch that dcn_backward needs.
+ *
+ * grad_x is a scatter (every tap adds to four pixels), accumulated in float32:
+ * for 16-bit data in a float32 copy of x's shape that the caller provides,
+ * N * H * W * C * 4 bytes; for float32 data in grad_x itself (0 bytes).
+ * Returns the byte count, or DCN_ERR_INVALID_ARG (< 0) for a negative or
+ * zero dimension (N < 0) or an unknown dtype.
+ */
+DCN_API long long dcn_backward_workspace_size(int N, int H, int W, int C, int dtype);
+
+/*
+ * dcn_backward - gradients of dcn_forward with respect to x, offset and mask.
+ *
+ * Defined by the same passages as dcn_forward, differentiated: "InternImage"
+ * ch.2 (the bilinear read is differentiable in the sampling position, which is
+ * how the offsets learn) and ch.3 / "DCNv4" "1. Remove Softmax" (the
+ * modulation with and without the softmax).  With go = grad_out:
+ *
+ *   grad_x[n][y][x][g*D+c]  = sum over taps (oy, ox, k) whose corner (y, x) is
+ *                             inside the map of m[k] * w_corner * go[n][oy][ox][g*D+c]
+ *   grad_offset[..][k][0]   = m[k] * sum_c go * dB/dpx,  [1]: dB/dpy, where
+ *                             dB/dpx = (1-b)(v01 - v00) + b(v11 - v10) and
+ *                             dB/dpy = (1-a)(v10 - v00) + a(v11 - v01), corners
+ *                             outside the map read 0; at an integer position the
+ *                             derivative is the one of the cell to the right/below
+ *   dL/dm[k]                = sum_c go * B(x, px, py)
+ *   grad_mask[..][k]        = dL/dm[k]                              (softmax_flag = 0)
+ *                           = m[k] * (dL/dm[k] - sum_j m[j] dL/dm[j])  (softmax_flag = 1:
+ *                             the gradient with respect to the logits)
+ *
+ * Arguments: x, offset, mask, softmax_flag, the sizes and dtype exactly as
+ * given to dcn_forward; grad_out [N][Ho][Wo][C]; outputs grad_x [N][H][W][C],
+ * grad_offset [N][Ho][Wo][G][K][2] and grad_mask [N][Ho][Wo][G][K], all in
+ * `dtype` and all overwritten.  `workspace` is caller-owned device scratch of
+ * at least dcn_backward_workspace_size() bytes, 16-byte aligned (ignored and
+ * may be NULL for float32); its contents on entry do not matter.
+ * Launches, in stream order: a zero fill of the float32 accumulator, the
+ * gradient kernel, and for 16-bit data the rounding of the accumulator into
+ * grad_x.  grad_x is a float32 sum whose order of additions is not fixed
+ * (hardware reductions), so its last bits may differ from run to run;
+ * grad_offset and grad_mask are deterministic.
+ * Limits: those of dcn_forward, plus: the shared-memory slice of one warp
+ * (the run's offsets, masks and their gradients: 6 * K * es * 32 / TPI bytes,
+ * and 4 * K * 32 / TPI more for softmax_flag = 1) at most 200 KiB
+ * (DCN_ERR_UNSUPPORTED otherwise; K <= 169 always fits).
+ * Errors: as dcn_forward, for every pointer; DCN_ERR_INVALID_ARG also when an
+ * output overlaps an input, another output or the workspace, or when
+ * workspace_bytes is too small; DCN_ERR_MISALIGNED for a workspace not
+ * aligned to 16 bytes.
+ */
+DCN_API int dcn_backward(const void* x, const void* offset, const void* mask,
+                 const void* grad_out, void* grad_x, void* grad_offset, void* grad_mask,
+                 void* workspace, long long workspace_bytes, int N, int H, int W, int C,
+                 int G, int kh, int kw, int stride, int pad, int dil, int softmax_flag,
+                 int dtype, void* stream);
+
+/*
+ * msda_backward_workspace_size - bytes of scratch that msda_backward needs:
+ * a float32 accumulator for grad_value, N * S * M * D * 4 bytes for 16-bit
+ * data, 0 for float32 (accumulated in grad_value itself); DCN_ERR_INVALID_ARG
+ * (< 0) for a bad dimension or dtype.
+ */
+DCN_API long long msda_backward_workspace_size(int N, int S, int M, int D, int dtype);
+
+/*
+ * msda_backward - gradients of msda_forward with respect to value,
+ * sampling_loc and attn_w.
+ *
+ * Defined by the passages of msda_forward, differentiated ("A learned
+ * location can fall between cells": the read is differentiable in the
+ * location).  With go = grad_out[n][q][h*D + c], x = u W_l - 1/2,
+ * y = v H_l - 1/2, a, b their fractional parts and A = attn_w[n][q][h][l][k]:
+ *
+ *   grad_value[n][start_l + r][h][c] += A * w_corner * go   for each corner r in the level
+ *   grad_loc[..][0] = A * W_l * sum_c go * ((1-b)(v01 - v00) + b(v11 - v10))
+ *   grad_loc[..][1] = A * H_l * sum_c go * ((1-a)(v10 - v00) + a(v11 - v01))
+ *   grad_attn[..]   = sum_c go * S_l(value, loc)
+ *
+ * Arguments: as msda_forward, plus S (value rows per batch item, equal to
+ * level_start[L-1] + H_{L-1} W_{L-1}), grad_out [N][Lq][M*D] and the outputs
+ * grad_value [N][S][M][D], grad_loc [N][Lq][M][L][K][2] and grad_attn
+ * [N][Lq][M][L][K], all in `dtype` and all overwritten.  `workspace` as for
+ * dcn_backward, of msda_backward_workspace_size() bytes.  grad_value's last
+ * bits depend on the order of hardware reductions; the others are
+ * deterministic.  Same launch sequence, limits and errors as msda_forward and
+ * dcn_backward (a warp's shared slice, 6 * L * K * es * 32 / TPI bytes, at
+ * most 200 KiB).
+ */
+DCN_API int msda_backward(const void* value, const int64_t* spatial_shapes,
+                  const int64_t* level_start, const void* sampling_loc, const void* attn_w,
+                  const void* grad_out, void* grad_value, void* grad_loc, void* grad_attn,
+                  void* workspace, long long workspace_bytes, int N, int S, int Lq, int M,
+                  int D, int L, int K, int dtype, void* stream);
 
 /* Output size of the deformable window: (in + 2 pad - dil (k - 1) - 1) / stride + 1,
  * or a value <= 0 when the window does not fit. */

@@ -27,12 +27,15 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return set(re.findall(r"^\s*DCN_API\s+(?:const\s+)?\w+\*?\s+\*?(\w+)\s*\(", text, flags=re.M))
+    return set(re.findall(r"^\s*DCN_API\s+(?:const\s+)?(?:\w+\s+)*?\w+\*?\s+\*?(\w+)\s*\(",
+                          text, flags=re.M))
 
 
 def test_header_declares_the_interface():
     names = declared_functions()
-    assert {"dcn_forward", "msda_forward", "dcn_status_string"} <= names
+    assert {"dcn_forward", "msda_forward", "dcn_backward", "msda_backward",
+            "dcn_backward_workspace_size", "msda_backward_workspace_size",
+            "dcn_status_string"} <= names
     assert names == set(dcnb.SIGNATURES), "binding signatures out of sync with dcn.h"
 
 
@@ -138,3 +141,93 @@ def test_binding_raises_with_status(lib):
         dcnb.dcn_forward(X, OFF, MASK, OUT, 1, 4, 4, 6, 4, 3, 3, 1, 1, 1, 0, F16, stream=0)
     assert e.value.status == dcnb.DCN_ERR_INVALID_ARG
     assert "invalid argument" in str(e.value)
+
+
+# more fake addresses for the backward's gradients and workspace
+GO, GX, GOFF, GMASK, WS = (0x7F0040000000, 0x7F0050000000, 0x7F0060000000, 0x7F0070000000,
+                           0x7F0080000000)
+
+
+def test_backward_workspace_sizes(lib):
+    assert dcnb.dcn_backward_workspace_size(2, 8, 8, 16, F16) == 2 * 8 * 8 * 16 * 4
+    assert dcnb.dcn_backward_workspace_size(2, 8, 8, 16, 2) == 2 * 8 * 8 * 16 * 4
+    assert dcnb.dcn_backward_workspace_size(2, 8, 8, 16, 0) == 0
+    assert dcnb.dcn_backward_workspace_size(0, 8, 8, 16, F16) == 0
+    assert dcnb.dcn_backward_workspace_size(2, 8, 8, 16, 9) == dcnb.DCN_ERR_INVALID_ARG
+    assert dcnb.dcn_backward_workspace_size(2, 0, 8, 16, F16) == dcnb.DCN_ERR_INVALID_ARG
+    assert dcnb.msda_backward_workspace_size(2, 100, 8, 32, F16) == 2 * 100 * 8 * 32 * 4
+    assert dcnb.msda_backward_workspace_size(2, 100, 8, 32, 0) == 0
+    assert dcnb.msda_backward_workspace_size(2, 0, 8, 32, F16) == dcnb.DCN_ERR_INVALID_ARG
+
+
+def call_dcn_bwd(lib, **kw):
+    args = dict(x=X, offset=OFF, mask=MASK, go=GO, gx=GX, goff=GOFF, gmask=GMASK, ws=WS,
+                ws_bytes=2 * 8 * 8 * 16 * 4, N=2, H=8, W=8, C=16, G=2, kh=3, kw=3, stride=1,
+                pad=1, dil=1, softmax_flag=0, dtype=F16, stream=None)
+    args.update(kw)
+    a = args
+    return lib.dcn_backward(a["x"], a["offset"], a["mask"], a["go"], a["gx"], a["goff"],
+                            a["gmask"], a["ws"], a["ws_bytes"], a["N"], a["H"], a["W"], a["C"],
+                            a["G"], a["kh"], a["kw"], a["stride"], a["pad"], a["dil"],
+                            a["softmax_flag"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(dtype=7), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(N=-1), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(C=15), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(softmax_flag=3), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(go=None), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(gx=None), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(gmask=None), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(ws=None), dcnb.DCN_ERR_INVALID_ARG),                 # 16-bit needs the workspace
+    (dict(ws_bytes=100), dcnb.DCN_ERR_INVALID_ARG),            # too small
+    (dict(ws=WS + 8), dcnb.DCN_ERR_MISALIGNED),                # not 16-byte aligned
+    (dict(gx=X), dcnb.DCN_ERR_INVALID_ARG),                    # grad_x aliases x
+    (dict(goff=GO + 64), dcnb.DCN_ERR_INVALID_ARG),            # overlaps grad_out
+    (dict(gmask=GOFF + 32), dcnb.DCN_ERR_INVALID_ARG),         # outputs overlap
+    (dict(ws=GX), dcnb.DCN_ERR_INVALID_ARG),                   # workspace overlaps grad_x
+    (dict(go=GO + 1), dcnb.DCN_ERR_MISALIGNED),
+    (dict(kh=25, kw=25, pad=12), dcnb.DCN_ERR_UNSUPPORTED),    # a warp's slice > 200 KiB
+    (dict(kh=21, kw=21, pad=10, softmax_flag=1), dcnb.DCN_ERR_UNSUPPORTED),
+    (dict(H=70000), dcnb.DCN_ERR_UNSUPPORTED),
+    (dict(N=0), dcnb.DCN_OK),
+    (dict(N=0, x=None, gx=None, ws=None), dcnb.DCN_OK),
+])
+def test_dcn_backward_validation(lib, change, status):
+    before = dcnb.dcn_launch_count()
+    assert call_dcn_bwd(lib, **change) == status
+    assert dcnb.dcn_launch_count() == before
+
+
+def call_msda_bwd(lib, **kw):
+    args = dict(value=X, shapes=OFF, starts=OFF + 1024, loc=MASK, attn=MASK + 2 ** 24, go=GO,
+                gv=GX, gl=GOFF, ga=GMASK, ws=WS, ws_bytes=2 * 3000 * 8 * 32 * 4, N=2, S=3000,
+                Lq=100, M=8, D=32, L=4, K=4, dtype=F16, stream=None)
+    args.update(kw)
+    a = args
+    return lib.msda_backward(a["value"], a["shapes"], a["starts"], a["loc"], a["attn"], a["go"],
+                             a["gv"], a["gl"], a["ga"], a["ws"], a["ws_bytes"], a["N"], a["S"],
+                             a["Lq"], a["M"], a["D"], a["L"], a["K"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(dtype=3), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(S=0), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(K=0), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(L=17), dcnb.DCN_ERR_UNSUPPORTED),
+    (dict(gv=None), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(gl=None), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(ws=None), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(ws_bytes=64), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(ws=WS + 4), dcnb.DCN_ERR_MISALIGNED),
+    (dict(gv=X), dcnb.DCN_ERR_INVALID_ARG),                    # grad_value aliases value
+    (dict(ga=GOFF + 64), dcnb.DCN_ERR_INVALID_ARG),            # overlaps grad_loc
+    (dict(gl=OFF), dcnb.DCN_ERR_INVALID_ARG),                  # overlaps the level table
+    (dict(starts=OFF + 1028), dcnb.DCN_ERR_MISALIGNED),
+    (dict(N=0, value=None, gv=None), dcnb.DCN_OK),
+])
+def test_msda_backward_validation(lib, change, status):
+    before = dcnb.dcn_launch_count()
+    assert call_msda_bwd(lib, **change) == status
+    assert dcnb.dcn_launch_count() == before
