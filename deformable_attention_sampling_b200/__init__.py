@@ -22,7 +22,9 @@ from ._binding import (  # noqa: F401
     SIGNATURES,
     DcnError,
     dcn,
+    STATIC_SCRATCH_BYTES,
     dcn_backward,
+    dcn_backward_static_scratch,
     dcn_backward_workspace_size,
     dcn_forward,
     dcn_grad,

@@ -31,6 +31,7 @@ SIGNATURES = {
     "msda_forward": (_I, [_VP] * 6 + [_I] * 7 + [_VP]),
     "dcn_backward_workspace_size": (_LL, [_I] * 5),
     "dcn_backward": (_I, [_VP] * 8 + [_LL] + [_I] * 12 + [_VP]),
+    "dcn_backward_static_scratch": (_I, [_VP] * 7 + [_I] * 12 + [_VP]),
     "msda_backward_workspace_size": (_LL, [_I] * 5),
     "msda_backward": (_I, [_VP] * 10 + [_LL] + [_I] * 8 + [_VP]),
     "dcn_output_size": (_I, [_I] * 5),
@@ -128,6 +129,21 @@ def dcn_backward(x, offset, mask, grad_out, grad_x, grad_offset, grad_mask, work
                                 workspace_bytes, N, H, W, C, G, kh, kw, stride, pad, dil,
                                 softmax_flag, dtype, _stream(stream)),
            "dcn_backward")
+
+
+# bytes of the library's static grad_x accumulator (DCN_STATIC_SCRATCH_BYTES)
+STATIC_SCRATCH_BYTES = 16 << 20
+
+
+def dcn_backward_static_scratch(x, offset, mask, grad_out, grad_x, grad_offset, grad_mask, N, H,
+                                W, C, G, kh, kw, stride, pad, dil, softmax_flag, dtype,
+                                stream=None):
+    """C dcn_backward_static_scratch (no workspace argument; the library's own
+    per-device accumulator); raises DcnError on a non-OK status."""
+    _check(_load().dcn_backward_static_scratch(
+        _ptr(x), _ptr(offset), _ptr(mask), _ptr(grad_out), _ptr(grad_x), _ptr(grad_offset),
+        _ptr(grad_mask), N, H, W, C, G, kh, kw, stride, pad, dil, softmax_flag, dtype,
+        _stream(stream)), "dcn_backward_static_scratch")
 
 
 def msda_backward_workspace_size(N, S, M, D, dtype):

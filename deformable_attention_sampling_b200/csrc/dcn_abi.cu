@@ -806,3 +806,74 @@ uint64_t dcn_launch_count(void) { return g_launches.load(std::memory_order_relax
 int dcn_version(void) { return 10000; }
 
 }  // extern "C"
+
+// ------------------------------------------- backward without caller scratch
+//
+// dcn_backward needs a float32 accumulator for grad_x of 16-bit data, and it
+// takes it from the caller.  Some callers have no device memory to hand over
+// at call time: a plain C host program that has no allocator of its own, or
+// code that must not allocate once it has started (a fixed device-memory
+// budget set at initialisation).  For them this file keeps one statically
+// sized accumulator per device, placed in the module's global memory when the
+// library's device code is loaded, and dcn_backward_static_scratch runs the
+// unchanged dcn_backward path with it.  Nothing is allocated per call.
+
+namespace {
+
+constexpr long long kStaticScratchBytes = DCN_STATIC_SCRATCH_BYTES;   // 16 MiB
+constexpr int kMaxScratchDevices = 64;
+
+__device__ __align__(256) float g_static_scratch[kStaticScratchBytes / 4];
+
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxScratchDevices] = {};
+
+// Device address of the static accumulator on the current device, looked up
+// (cudaGetSymbolAddress) the first time a device asks and cached after that.
+int static_scratch(void** out) {
+    int device = 0;
+    cudaError_t err = cudaGetDevice(&device);
+    if (err != cudaSuccess) {
+        g_last_cuda_error = (int)err;
+        (void)cudaGetLastError();
+        return DCN_ERR_CUDA;
+    }
+    if (device < 0 || device >= kMaxScratchDevices) return DCN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_ptr[device] == nullptr) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (err != cudaSuccess || p == nullptr) {
+            g_last_cuda_error = (int)(err != cudaSuccess ? err : cudaErrorInvalidSymbol);
+            (void)cudaGetLastError();
+            return DCN_ERR_CUDA;
+        }
+        g_scratch_ptr[device] = p;
+    }
+    *out = g_scratch_ptr[device];
+    return DCN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dcn_backward_static_scratch(const void* x, const void* offset, const void* mask,
+                                const void* grad_out, void* grad_x, void* grad_offset,
+                                void* grad_mask, int N, int H, int W, int C, int G, int kh,
+                                int kw, int stride, int pad, int dil, int softmax_flag,
+                                int dtype, void* stream) {
+    const long long need = dcn_backward_workspace_size(N, H, W, C, dtype);
+    if (need < 0) return DCN_ERR_INVALID_ARG;
+    if (need > kStaticScratchBytes) return DCN_ERR_UNSUPPORTED;
+    void* ws = nullptr;
+    if (need > 0) {
+        const int rc = static_scratch(&ws);
+        if (rc != DCN_OK) return rc;
+    }
+    return dcn_backward(x, offset, mask, grad_out, grad_x, grad_offset, grad_mask, ws,
+                        need > 0 ? kStaticScratchBytes : 0, N, H, W, C, G, kh, kw, stride, pad,
+                        dil, softmax_flag, dtype, stream);
+}
+
+}  // extern "C"

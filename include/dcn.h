@@ -187,6 +187,38 @@ DCN_API int dcn_backward(const void* x, const void* offset, const void* mask,
                  int G, int kh, int kw, int stride, int pad, int dil, int softmax_flag,
                  int dtype, void* stream);
 
+/* Size of the library's own static grad_x accumulator (one per device). */
+#define DCN_STATIC_SCRATCH_BYTES (16LL << 20)
+
+/*
+ * dcn_backward_static_scratch - dcn_backward with the library's own scratch.
+ *
+ * The pages describe no counterpart: this is an interface convenience, not a
+ * step of the method.  It is for callers that cannot hand dcn_backward a
+ * workspace: a C host program with no device allocator of its own at call
+ * time, or code that must not allocate once it has started (a fixed memory
+ * budget).  Arguments, results, launches and errors are those of
+ * dcn_backward, without `workspace` / `workspace_bytes`: for 16-bit data the
+ * float32 grad_x accumulator is a statically sized array in the library's
+ * device code (DCN_STATIC_SCRATCH_BYTES per device, reserved when the
+ * library's device code is loaded on that device).  No call allocates.
+ *   - Limit: N * H * W * C * 4 <= DCN_STATIC_SCRATCH_BYTES for f16 / bf16
+ *     (N * H * W * C <= 4194304); beyond it DCN_ERR_UNSUPPORTED, nothing
+ *     launched.  float32 data needs no scratch and has no such limit.
+ *   - The first call on a device (with 16-bit data) looks up the array's
+ *     device address with cudaGetSymbolAddress, with that device current,
+ *     and caches it; a failure returns DCN_ERR_CUDA.  Make that first call
+ *     before any stream capture on the device.
+ *   - The accumulator is zero-filled by every call (it needs no clearing
+ *     between calls), but there is one per device: calls whose work overlaps
+ *     in time on one device (other streams, other host threads) race on it
+ *     and give wrong grad_x.  Calls issued in order on one stream are safe.
+ */
+DCN_API int dcn_backward_static_scratch(const void* x, const void* offset, const void* mask,
+                 const void* grad_out, void* grad_x, void* grad_offset, void* grad_mask,
+                 int N, int H, int W, int C, int G, int kh, int kw, int stride, int pad,
+                 int dil, int softmax_flag, int dtype, void* stream);
+
 /*
  * msda_backward_workspace_size - bytes of scratch that msda_backward needs:
  * a float32 accumulator for grad_value, N * S * M * D * 4 bytes for 16-bit
