@@ -47,19 +47,21 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic of the timed kernel from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum per launch, headline workload), with the hash of the
-# kernel sources it was taken on; reported as null once the sources change.
+# forward kernel's sources it was taken on; reported as null once they change.
 NCU_TRAFFIC = {
-    "source_sha256": "dbbd5eda7ae979c14fa9dde969cff6742468141b972e1367bca0742794417906",
-    "bytes_per_launch": 69166336 + 3505408,   # DRAM read + write, one headline launch
+    "source_sha256": "6153b12ff5da32abec3aa2b88a07b2211c9d6bd6b43e0667a7e965e94f9e7a64",
+    "bytes_per_launch": 69196544 + 3538944,   # DRAM read + write, one headline launch
 }
 
-KERNEL_SOURCES = [
+# What the forward DCN launch depends on: its device code, and in the C
+# interface the tile choice, the kernel dispatch and dcn_forward itself.
+FORWARD_SOURCES = [
     "deformable_attention_sampling_b200/csrc/common.cuh",
     "deformable_attention_sampling_b200/csrc/dcn_fwd.cuh",
-    "deformable_attention_sampling_b200/csrc/msda_fwd.cuh",
-    "deformable_attention_sampling_b200/csrc/dcn_abi.cu",
-    "include/dcn.h",
 ]
+FORWARD_ABI = "deformable_attention_sampling_b200/csrc/dcn_abi.cu"
+FORWARD_ABI_SPANS = [("struct TileShape {", "// ---------------------------------------------------------------- MSDA"),
+                     ("int dcn_forward(", "int msda_forward(")]
 
 
 def log(*a):
@@ -68,9 +70,14 @@ def log(*a):
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in FORWARD_SOURCES:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
+    with open(os.path.join(ROOT, FORWARD_ABI)) as f:
+        text = f.read()
+    for begin, end in FORWARD_ABI_SPANS:
+        i = text.index(begin)
+        h.update(text[i:text.index(end, i)].encode())
     return h.hexdigest()
 
 

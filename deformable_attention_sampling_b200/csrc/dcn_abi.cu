@@ -256,18 +256,23 @@ const void* msda_kernel_vb(int vb) {
 
 // ------------------------------------------------------------ backward ---
 
-template <typename T, int VB>
+template <typename T, int VB, bool PAIR = false>
 const void* dcn_bwd_kernel_for(int softmax, int kh, int kw) {
     using namespace dcnb;
     if (kh == 3 && kw == 3)
-        return softmax ? (const void*)dcn_bwd_kernel<T, VB, true, 3>
-                       : (const void*)dcn_bwd_kernel<T, VB, false, 3>;
-    return softmax ? (const void*)dcn_bwd_kernel<T, VB, true>
-                   : (const void*)dcn_bwd_kernel<T, VB, false>;
+        return softmax ? (const void*)dcn_bwd_kernel<T, VB, true, 3, PAIR>
+                       : (const void*)dcn_bwd_kernel<T, VB, false, 3, PAIR>;
+    return softmax ? (const void*)dcn_bwd_kernel<T, VB, true, 0, PAIR>
+                   : (const void*)dcn_bwd_kernel<T, VB, false, 0, PAIR>;
 }
 
 template <typename T>
-const void* dcn_bwd_kernel_vb(int vb, int kh, int kw, int softmax) {
+const void* dcn_bwd_kernel_vb(int vb, int kh, int kw, int softmax, int pair) {
+    if (pair) {   // 8 channels per lane
+        if (vb == 8 * (int)sizeof(T))
+            return dcn_bwd_kernel_for<T, 8 * sizeof(T), true>(softmax, kh, kw);
+        return nullptr;
+    }
     switch (vb) {
         case 32: return dcn_bwd_kernel_for<T, 32>(softmax, kh, kw);
         case 16: return dcn_bwd_kernel_for<T, 16>(softmax, kh, kw);
@@ -282,8 +287,12 @@ const void* dcn_bwd_kernel_vb(int vb, int kh, int kw, int softmax) {
 }
 
 template <typename T>
-const void* msda_bwd_kernel_vb(int vb) {
+const void* msda_bwd_kernel_vb(int vb, int pair) {
     using namespace dcnb;
+    if (pair) {   // 8 channels per lane
+        if (vb == 8 * (int)sizeof(T)) return (const void*)msda_bwd_kernel<T, 8 * sizeof(T), true>;
+        return nullptr;
+    }
     switch (vb) {
         case 32: return (const void*)msda_bwd_kernel<T, 32>;
         case 16: return (const void*)msda_bwd_kernel<T, 16>;
@@ -306,6 +315,23 @@ int pick_red_vec(const void* acc, long long pix_floats, int cpt) {
             return rv;
     }
     return 1;
+}
+
+// Per-lane vector width of a backward kernel.  Where a group's (head's)
+// channels split into an even number of 8-channel lanes and the accumulator's
+// 32-byte sectors line up with them, 8 channels per lane (one float32 sector)
+// so that lane pairs reduce whole sectors (*pair = 1); otherwise the forward's
+// widest vector.
+int pick_bwd_vector_bytes(int es, int D, uintptr_t bases, const void* acc,
+                          long long pix_floats, int* pair) {
+    *pair = 0;
+    const int vb8 = 8 * es;
+    if (D % 16 == 0 && bases % (uintptr_t)vb8 == 0 && (uintptr_t)acc % 32 == 0 &&
+        pix_floats % 8 == 0) {
+        *pair = 1;
+        return vb8;
+    }
+    return pick_vector_bytes(es, D, bases);
 }
 
 // The accumulator set-up and wrap-up launches around a backward kernel.
@@ -591,7 +617,10 @@ int dcn_backward(const void* x, const void* offset, const void* mask, const void
         }
     }
 
-    const int vb = pick_vector_bytes(es, D, (uintptr_t)x | (uintptr_t)grad_out);
+    float* acc = dtype == DCN_F32 ? static_cast<float*>(grad_x) : static_cast<float*>(workspace);
+    int pair = 0;
+    const int vb = pick_bwd_vector_bytes(es, D, (uintptr_t)x | (uintptr_t)grad_out, acc, C,
+                                         &pair);
     if (vb == 0) return DCN_ERR_MISALIGNED;
     const int cpt = vb / es;
     const int tpi = D / cpt;
@@ -618,7 +647,6 @@ int dcn_backward(const void* x, const void* offset, const void* mask, const void
     const long long num_tiles = tiles_per_image * N;
     if (num_tiles > kInt31) return DCN_ERR_UNSUPPORTED;
 
-    float* acc = dtype == DCN_F32 ? static_cast<float*>(grad_x) : static_cast<float*>(workspace);
     dcnb::DcnBwdArgs b;
     dcnb::DcnArgs& a = b.f;
     a.x = x;
@@ -664,9 +692,11 @@ int dcn_backward(const void* x, const void* offset, const void* mask, const void
 
     const void* fn = nullptr;
     switch (dtype) {
-        case DCN_F32: fn = dcn_bwd_kernel_vb<float>(vb, kh, kw, softmax_flag); break;
-        case DCN_F16: fn = dcn_bwd_kernel_vb<__half>(vb, kh, kw, softmax_flag); break;
-        case DCN_BF16: fn = dcn_bwd_kernel_vb<__nv_bfloat16>(vb, kh, kw, softmax_flag); break;
+        case DCN_F32: fn = dcn_bwd_kernel_vb<float>(vb, kh, kw, softmax_flag, pair); break;
+        case DCN_F16: fn = dcn_bwd_kernel_vb<__half>(vb, kh, kw, softmax_flag, pair); break;
+        case DCN_BF16:
+            fn = dcn_bwd_kernel_vb<__nv_bfloat16>(vb, kh, kw, softmax_flag, pair);
+            break;
         default: break;
     }
     if (!fn) return DCN_ERR_UNSUPPORTED;
@@ -729,7 +759,11 @@ int msda_backward(const void* value, const int64_t* spatial_shapes, const int64_
         }
     }
 
-    const int vb = pick_vector_bytes(es, D, (uintptr_t)value | (uintptr_t)grad_out);
+    float* acc =
+        dtype == DCN_F32 ? static_cast<float*>(grad_value) : static_cast<float*>(workspace);
+    int pair = 0;
+    const int vb = pick_bwd_vector_bytes(es, D, (uintptr_t)value | (uintptr_t)grad_out, acc,
+                                         (long long)M * D, &pair);
     if (vb == 0) return DCN_ERR_MISALIGNED;
     const int cpt = vb / es;
     const int tpi = D / cpt;
@@ -739,8 +773,6 @@ int msda_backward(const void* value, const int64_t* spatial_shapes, const int64_
     if (slice > kMaxBwdSliceBytes || slice * dcnb::kMsdaWarps > kMaxBwdSmemBytes)
         return DCN_ERR_UNSUPPORTED;
 
-    float* acc =
-        dtype == DCN_F32 ? static_cast<float*>(grad_value) : static_cast<float*>(workspace);
     const long long acc_elems = (long long)N * S * M * D;
     dcnb::MsdaBwdArgs b;
     dcnb::MsdaArgs& a = b.f;
@@ -772,9 +804,9 @@ int msda_backward(const void* value, const int64_t* spatial_shapes, const int64_
 
     const void* fn = nullptr;
     switch (dtype) {
-        case DCN_F32: fn = msda_bwd_kernel_vb<float>(vb); break;
-        case DCN_F16: fn = msda_bwd_kernel_vb<__half>(vb); break;
-        case DCN_BF16: fn = msda_bwd_kernel_vb<__nv_bfloat16>(vb); break;
+        case DCN_F32: fn = msda_bwd_kernel_vb<float>(vb, pair); break;
+        case DCN_F16: fn = msda_bwd_kernel_vb<__half>(vb, pair); break;
+        case DCN_BF16: fn = msda_bwd_kernel_vb<__nv_bfloat16>(vb, pair); break;
         default: break;
     }
     if (!fn) return DCN_ERR_UNSUPPORTED;

@@ -20,8 +20,11 @@
 // with P = 0 for corners outside the map, and reduces the three over the
 // item's threads with warp shuffles.  The grad_x scatter goes to a float32
 // accumulator with vector reductions (red.global.add.v4.f32: 16 bytes per
-// instruction, resolved in L2); the caller's launch sequence zeroes the
-// accumulator first and, for 16-bit data, rounds it into grad_x afterwards.
+// instruction, resolved in L2), issued so that each instruction of a lane
+// pair fills whole 32-byte sectors when an item has an even number of 8-channel
+// lanes (the reduction throughput of L2 is per sector); the caller's launch
+// sequence zeroes the accumulator first and, for 16-bit data, rounds it into
+// grad_x afterwards.
 // grad_offset and grad_mask of a run are collected in the warp's shared slice
 // and written with coalesced stores.
 #pragma once
@@ -30,7 +33,7 @@
 
 namespace dcnb {
 
-constexpr int kDcnBwdMaxWarps = 16;
+constexpr int kDcnBwdMaxWarps = 16;   // 128 registers: 16 warps per SM
 constexpr int kDcnBwdMaxThreads = 32 * kDcnBwdMaxWarps;
 
 struct DcnBwdArgs {
@@ -102,6 +105,43 @@ __device__ __forceinline__ void warp_stage_out(T* dst, const T* src, int elems, 
         unsigned short* d = reinterpret_cast<unsigned short*>(dst);
         for (int i = lane; i < (nbytes >> 1); i += 32) d[i] = s[i];
     }
+}
+
+// Sector-paired scatter (CPT = 8, an even number of lanes per item).  L2
+// resolves reductions per 32-byte sector, so two 16-byte reductions to one
+// sector cost as much as two full ones.  The two lanes 2j, 2j+1 of an item own
+// 8 channels each (one float32 sector each); in the first instruction both
+// add to lane 2j's sector (lane 2j its channels 0-3, lane 2j+1 lane 2j's
+// channels 4-7), in the second both add to lane 2j+1's sector.  The values a
+// lane adds are fixed per item: v1 / v2 and the float offsets d1 / d2 come
+// from pair_setup, so the scatter itself is branch-free.
+struct PairScatter {
+    float v1[4], v2[4];
+    int d1, d2;
+};
+
+// Every lane of the warp must call it (one shuffle exchange per item).
+__device__ __forceinline__ PairScatter pair_setup(const float* go, int chunk) {
+    PairScatter ps;
+    const bool odd = chunk & 1;
+    float recv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)   // the partner's half that this lane adds
+        recv[i] = __shfl_xor_sync(0xffffffffu, odd ? go[i] : go[4 + i], 1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        ps.v1[i] = odd ? recv[i] : go[i];        // lane 2j's sector
+        ps.v2[i] = odd ? go[4 + i] : recv[i];    // lane 2j+1's sector
+    }
+    ps.d1 = odd ? -4 : 0;
+    ps.d2 = odd ? 4 : 8;
+    return ps;
+}
+
+// p = this lane's first channel in the accumulator
+__device__ __forceinline__ void scatter_pair(float* p, float coef, const PairScatter& ps) {
+    red_add4(p + ps.d1, coef * ps.v1[0], coef * ps.v1[1], coef * ps.v1[2], coef * ps.v1[3]);
+    red_add4(p + ps.d2, coef * ps.v2[0], coef * ps.v2[1], coef * ps.v2[2], coef * ps.v2[3]);
 }
 
 // sum_i a[i] * b[i] for i < CPT (two lanes per FFMA2)
@@ -188,7 +228,9 @@ __host__ __device__ inline BwdSlice bwd_slice(int run_items, int K, int es, bool
     return s;
 }
 
-template <typename T, int VB, bool SOFTMAX, int KF = 0>
+// PAIR: the sector-paired scatter (CPT = 8, an even number of lanes per item),
+// chosen on the host; otherwise plain vector reductions of width b.red_vec.
+template <typename T, int VB, bool SOFTMAX, int KF = 0, bool PAIR = false>
 __global__ void __launch_bounds__(kDcnBwdMaxThreads, 1) dcn_bwd_kernel(const DcnBwdArgs b) {
     constexpr int UNROLL = KF ? KF * KF : 1;
     constexpr int CPT = VB / (int)sizeof(T);
@@ -271,6 +313,9 @@ __global__ void __launch_bounds__(kDcnBwdMaxThreads, 1) dcn_bwd_kernel(const Dcn
                 for (int i = 0; i < CPT; ++i) go[i] = 0.f;
             }
         }
+        static_assert(!PAIR || CPT == 8, "the paired scatter needs 8 channels per lane");
+        PairScatter ps;
+        if constexpr (PAIR) ps = pair_setup(go, chunk);
 
         float zmax = 0.f, inv_sum = 1.f;
         if constexpr (SOFTMAX) {
@@ -325,8 +370,12 @@ __global__ void __launch_bounds__(kDcnBwdMaxThreads, 1) dcn_bwd_kernel(const Dcn
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const float wc = (c & 1 ? wx1 : wx0) * (c & 2 ? wy1 : wy0);
-                if (active && ((cur.valid >> c) & 1u))
-                    scatter_scaled<CPT>(gxb + cur.off[c] / es, m * wc, go, b.red_vec);
+                if (active && ((cur.valid >> c) & 1u)) {
+                    if constexpr (PAIR)
+                        scatter_pair(gxb + cur.off[c] / es, m * wc, ps);
+                    else
+                        scatter_scaled<CPT>(gxb + cur.off[c] / es, m * wc, go, b.red_vec);
+                }
             }
             float gm = wy0 * (wx0 * P[0] + wx1 * P[1]) + wy1 * (wx0 * P[2] + wx1 * P[3]);
             float da = wy0 * (P[1] - P[0]) + wy1 * (P[3] - P[2]);

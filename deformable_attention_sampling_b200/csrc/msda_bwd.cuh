@@ -12,7 +12,9 @@
 // tap each thread forms the corner dot products P_c = sum over its channels
 // of go * value_corner and combines them as the DCN backward does; the three
 // per-tap sums are reduced over the item's threads with shuffles.  grad_value
-// goes to a float32 accumulator through vector reductions in L2.
+// goes to a float32 accumulator through vector reductions in L2, whole
+// 32-byte sectors per lane pair where the channel split allows (as in the
+// DCN backward).
 #pragma once
 
 #include "dcn_bwd.cuh"
@@ -82,7 +84,10 @@ __host__ __device__ inline MsdaBwdSlice msda_bwd_slice(int run_items, int LK, in
     return s;
 }
 
-template <typename T, int VB>
+// PAIR: the sector-paired scatter (CPT = 8, an even number of lanes per item).
+// 128 registers: four 4-warp CTAs per SM (measured faster than a register cap
+// that fits six, which spills).
+template <typename T, int VB, bool PAIR = false>
 __global__ void __launch_bounds__(kMsdaThreads, 4) msda_bwd_kernel(const MsdaBwdArgs b) {
     constexpr int CPT = VB / (int)sizeof(T);
     constexpr int NW = VB >= 4 ? VB / 4 : 1;
@@ -151,6 +156,9 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_bwd_kernel(const MsdaBwd
                 for (int i = 0; i < CPT; ++i) go[i] = 0.f;
             }
         }
+        static_assert(!PAIR || CPT == 8, "the paired scatter needs 8 channels per lane");
+        PairScatter ps;
+        if constexpr (PAIR) ps = pair_setup(go, chunk);
 
         uint32_t v[4][NW];
         int nl = 0, nt = 0;
@@ -185,8 +193,12 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_bwd_kernel(const MsdaBwd
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const float wc = (c & 1 ? wx1 : wx0) * (c & 2 ? wy1 : wy0);
-                if (active && ((cur.valid >> c) & 1u))
-                    scatter_scaled<CPT>(gvb + cur.off[c], A * wc, go, b.red_vec);
+                if (active && ((cur.valid >> c) & 1u)) {
+                    if constexpr (PAIR)
+                        scatter_pair(gvb + cur.off[c], A * wc, ps);
+                    else
+                        scatter_scaled<CPT>(gvb + cur.off[c], A * wc, go, b.red_vec);
+                }
             }
             float gs = wy0 * (wx0 * P[0] + wx1 * P[1]) + wy1 * (wx0 * P[2] + wx1 * P[3]);
             float da = wy0 * (P[1] - P[0]) + wy1 * (P[3] - P[2]);
