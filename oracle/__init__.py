@@ -5,8 +5,9 @@ CUDA library is checked against.  Only the test suite, the smoke check and the
 benchmark's CPU-baseline leg may import it; the product path never does, and
 it imports nothing from the product package.
 
-`dcn_forward_ref` and `msda_forward_ref` call the C loop nests in
-dcn_oracle.c through ctypes.  Inputs may be numpy arrays or torch CPU tensors
+`dcn_forward_ref`, `msda_forward_ref`, their backward twins and
+`dynconv_forward_ref` (the ContMix core) call the C loop nests in dcn_oracle.c
+through ctypes.  Inputs may be numpy arrays or torch CPU tensors
 in any floating dtype; each value is converted exactly to float64 before the
 arithmetic (every fp16, bf16 and fp32 value is representable in float64).
 
@@ -39,6 +40,8 @@ def bind(lib):
     lib.oracle_dcn_backward.restype = ctypes.c_int
     lib.oracle_msda_backward.argtypes = [dp, lp, lp, dp, dp, dp, dp, dp, dp] + [L] * 7
     lib.oracle_msda_backward.restype = ctypes.c_int
+    lib.oracle_dynconv_forward.argtypes = [dp, dp, dp] + [L] * 6 + [ctypes.c_int]
+    lib.oracle_dynconv_forward.restype = ctypes.c_int
     return lib
 
 
@@ -168,3 +171,22 @@ def msda_backward_ref(value, spatial_shapes, level_start, loc, attn, grad_out):
     if rc != 0:
         raise ValueError("oracle_msda_backward rejected its arguments")
     return gv, gl, ga
+
+
+def dynconv_forward_ref(x, weights, K, softmax_flag=1, groups=None):
+    """float64 dynamic local aggregation (ContMix core).
+
+    x [N, H, W, C], weights [N, H, W, G, K*K] (tap ky * K + kx) -> out
+    [N, H, W, C] float64; K odd.  G is taken from weights.shape[3] unless given.
+    """
+    x = _as_f64(x)
+    weights = _as_f64(weights)
+    N, H, W, C = x.shape
+    G = groups if groups is not None else weights.shape[3]
+    assert weights.size == N * H * W * G * K * K, "weights has the wrong size"
+    out = np.zeros((N, H, W, C), dtype=np.float64)
+    rc = _load().oracle_dynconv_forward(_ptr(x), _ptr(weights), _ptr(out), N, H, W, C, G, K,
+                                        int(softmax_flag))
+    if rc != 0:
+        raise ValueError("oracle_dynconv_forward rejected its arguments")
+    return out

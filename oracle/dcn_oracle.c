@@ -25,6 +25,11 @@
  *        (1-|x-i|)+ (1-|y-j|)+ over the four floor/ceil neighbours, zero
  *        outside, no clamping, no renormalisation) and helper 3 (h_m = sum over
  *        levels and points of A_mlk times the sampled value).
+ *   [P5] "OverLoCK" note, "ContMix: Put the Whole Image into the Kernel"
+ *        (steps 4-5: a softmax turns each location's K^2 numbers into its own
+ *        K x K kernel per channel group, which is applied to the zero-padded
+ *        K x K neighbourhood of that group's channels; the note's snippet
+ *        unfolds with padding K // 2, so taps are row-major, ky * K + kx).
  *
  * Readings where the sources are silent (each also listed in the design notes):
  *   - tap index k = ix * kh + iy for a kh x kw window (the grid R of [P1] ch.1 is
@@ -404,5 +409,61 @@ int oracle_msda_backward(const double *value, const long long *shapes,
             }
         }
     }
+    return 0;
+}
+
+/*
+ * Dynamic local aggregation (the ContMix core), [P5] "ContMix" steps 4-5.
+ * x [N][H][W][C], w [N][H][W][G][K*K] (tap t = ky * K + kx), out [N][H][W][C]:
+ *   out[n][y][x][g*D + c] = sum_{ky, kx} A[t] * x[n][y + ky - K/2][x + kx - K/2][g*D + c]
+ * with 0 outside the map, A = softmax over the K*K weights of the location and
+ * group (softmax_flag = 1) or the weights as given (0).  K must be odd (the
+ * output keeps the input size).
+ */
+int oracle_dynconv_forward(const double *x, const double *w, double *out, long N, long H,
+                           long W, long C, long G, long K, int softmax_flag)
+{
+    if (N < 0 || H <= 0 || W <= 0 || C <= 0 || G <= 0 || C % G != 0 || K <= 0 || K % 2 != 1)
+        return -1;
+    long D = C / G;
+    long KK = K * K;
+    long r = K / 2;
+    double *A = (double *)malloc(sizeof(double) * (size_t)KK);
+    if (!A)
+        return -1;
+    for (long n = 0; n < N; ++n)
+    for (long y = 0; y < H; ++y)
+    for (long xx = 0; xx < W; ++xx)
+    for (long g = 0; g < G; ++g) {
+        const double *wt = w + (((n * H + y) * W + xx) * G + g) * KK;
+        if (softmax_flag) {
+            double zmax = wt[0];
+            for (long t = 1; t < KK; ++t)
+                if (wt[t] > zmax)
+                    zmax = wt[t];
+            double sum = 0.0;
+            for (long t = 0; t < KK; ++t) {
+                A[t] = exp(wt[t] - zmax);
+                sum += A[t];
+            }
+            for (long t = 0; t < KK; ++t)
+                A[t] = A[t] / sum;
+        } else {
+            for (long t = 0; t < KK; ++t)
+                A[t] = wt[t];
+        }
+        for (long c = 0; c < D; ++c) {
+            double acc = 0.0;
+            for (long ky = 0; ky < K; ++ky)
+            for (long kx = 0; kx < K; ++kx) {
+                long sy = y + ky - r, sx = xx + kx - r;
+                if (sy < 0 || sy >= H || sx < 0 || sx >= W)
+                    continue;
+                acc += A[ky * K + kx] * x[((n * H + sy) * W + sx) * C + g * D + c];
+            }
+            out[((n * H + y) * W + xx) * C + g * D + c] = acc;
+        }
+    }
+    free(A);
     return 0;
 }

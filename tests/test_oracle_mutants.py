@@ -17,6 +17,7 @@ import pytest
 import oracle
 from oracle import build as oracle_build
 from tests import test_oracle_backward_pins as bwd
+from tests import test_oracle_dynconv_pins as dyn
 from tests import test_oracle_pins as pins
 from tests.conftest import read_golden
 
@@ -60,6 +61,25 @@ MUTANTS_BWD = {
     "msda grad_value misses A": ("double ga = go * A;", "double ga = go;"),
     "msda grad_attn": ("grad_attn[t] += go * sample;", "grad_attn[t] += sample;"),
 }
+
+# mistakes planted in the dynamic local aggregation (ContMix core)
+MUTANTS_DYN = {
+    "dyn taps column-major": ("acc += A[ky * K + kx] * x[", "acc += A[kx * K + ky] * x["),
+    "dyn window not centred": ("long sy = y + ky - r, sx = xx + kx - r;",
+                               "long sy = y + ky - r, sx = xx + kx;"),
+    "dyn softmax not normalised": ("A[t] = A[t] / sum;", "A[t] = A[t];"),
+    "dyn group channel offset": ("* C + g * D + c];\n            }", "* C + c];\n            }"),
+    "dyn lower bound off by one": ("if (sy < 0 || sy >= H || sx < 0 || sx >= W)",
+                                   "if (sy < 0 || sy >= H || sx < 1 || sx >= W)"),
+    "dyn weights of the wrong group": ("const double *wt = w + (((n * H + y) * W + xx) * G + g) * KK;",
+                                       "const double *wt = w + (((n * H + y) * W + xx) * G) * KK;"),
+}
+
+PIN_TESTS_DYN = [
+    (dyn.test_matches_unfold_formulation, [dict(case=c) for c in dyn.CASES[:3]]),
+    (dyn.test_one_hot_weights_copy_a_shifted_map, [{}]),
+    (dyn.test_equal_logits_give_the_zero_padded_box_mean, [dict(K=3)]),
+]
 
 PIN_TESTS_BWD = [
     (bwd.test_dcn_grad_x_is_the_adjoint, [dict(case=c) for c in bwd.DCN_CASES[:2]]),
@@ -109,6 +129,7 @@ def _failures(battery=PIN_TESTS):
 def test_real_oracle_passes_the_battery():
     assert _failures() == []
     assert _failures(PIN_TESTS_BWD) == []
+    assert _failures(PIN_TESTS_DYN) == []
 
 
 def _install_mutant(original, planted, tmp_path, monkeypatch):
@@ -125,6 +146,12 @@ def _install_mutant(original, planted, tmp_path, monkeypatch):
 def test_backward_mutant_is_caught(name, tmp_path, monkeypatch):
     _install_mutant(*MUTANTS_BWD[name], tmp_path, monkeypatch)
     assert _failures(PIN_TESTS_BWD), f"no backward pin caught the mutant '{name}'"
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS_DYN))
+def test_dynconv_mutant_is_caught(name, tmp_path, monkeypatch):
+    _install_mutant(*MUTANTS_DYN[name], tmp_path, monkeypatch)
+    assert _failures(PIN_TESTS_DYN), f"no dynamic-kernel pin caught the mutant '{name}'"
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
