@@ -192,6 +192,21 @@ def on_chip_roofline(w, ms_per_launch, sampler, device):
                           f" x {sms} SMs x {mhz} MHz"}
 
 
+def fma_roofline(w, ms_per_launch, sampler, device):
+    """The arithmetic side of the ContMix core: one float32 FMA per (location,
+    tap, channel), against the SMs' float32 FMA rate (128 lanes per SM per
+    clock) at the median SM clock sampled during the timed region."""
+    fmas = w.taps() * w.D
+    achieved = 2 * fmas / (ms_per_launch * 1e-3) / 1e12
+    clocks = sampler.summary()
+    mhz = clocks["sm_mhz"] or clocks["sm_max_mhz"] or 1965
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    peak = 2 * 128 * sms * mhz * 1e6 / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "fma_per_launch": fmas,
+            "peak_basis": f"128 FP32 FMA lanes x {sms} SMs x {mhz} MHz"}
+
+
 # ------------------------------------------------------------------ runners
 
 class DcnRunner:
@@ -364,7 +379,50 @@ class MsdaBwdRunner(MsdaRunner):
         return self.w.backward_bytes()
 
 
+class DynRunner:
+    """One step = one dynconv_forward call (the ContMix core)."""
+    kernel = "dynconv_fwd_kernel"
+
+    def __init__(self, w, seed, device):
+        import deformable_attention_sampling_b200 as dcnb
+        self.dcnb = dcnb
+        self.w = w
+        self.host = gen.dynconv_inputs(w, seed=seed)
+        self.device = device
+        self.code = gen.DTYPE_CODES[w.dtype]
+        self.lib = dcnb.library()
+
+    def alloc_set(self):
+        d = {k: v.to(self.device) for k, v in self.host.items()}
+        d["out"] = torch.empty_like(d["x"])
+        return d
+
+    def launcher(self, s, stream):
+        w, lib = self.w, self.lib
+        args = (s["x"].data_ptr(), s["weights"].data_ptr(), s["out"].data_ptr(), w.N, w.H, w.W,
+                w.C, w.G, w.K, w.softmax_flag, self.code, stream)
+
+        def go():
+            st = lib.dynconv_forward(*args)
+            if st != 0:
+                raise self.dcnb.DcnError(st, "dynconv_forward")
+        return go
+
+    def inputs_of(self, s):
+        return [(s["x"], self.host["x"]), (s["weights"], self.host["weights"])]
+
+    def outputs_of(self, s):
+        return [s["out"]]
+
+    def bytes_per_step(self):
+        return self.w.compulsory_bytes()
+
+
 def make_runner(w, seed, device, backward=False):
+    if isinstance(w, gen.DynWorkload):
+        if backward:
+            raise SystemExit("--pass backward is not offered for the ContMix workloads")
+        return DynRunner(w, seed, device)
     dcn = isinstance(w, gen.DcnWorkload)
     if backward:
         return (DcnBwdRunner if dcn else MsdaBwdRunner)(w, seed, device)
@@ -388,6 +446,10 @@ def oracle_step(w, seed, backward=False):
         t = time.perf_counter()
         oracle.msda_backward_ref(inp["value"], inp["spatial_shapes"], inp["level_start"],
                                  inp["loc"], inp["attn"], go)
+    elif isinstance(w, gen.DynWorkload):
+        inp = gen.dynconv_inputs(w, seed=seed)
+        t = time.perf_counter()
+        oracle.dynconv_forward_ref(inp["x"], inp["weights"], w.K, w.softmax_flag)
     elif isinstance(w, gen.DcnWorkload):
         inp = gen.dcn_inputs(w, seed=seed)
         t = time.perf_counter()
@@ -404,7 +466,7 @@ def oracle_step(w, seed, backward=False):
 def sample_of(w, n_images):
     """A bounded sample of workload w with the same per-tap work: fewer batch
     items (DCN) or fewer queries (MSDA)."""
-    if isinstance(w, gen.DcnWorkload):
+    if isinstance(w, (gen.DcnWorkload, gen.DynWorkload)):
         return gen.scaled(w, N=max(1, min(w.N, n_images)))
     return gen.scaled(w, N=1, Lq=max(1, min(w.queries, n_images * 64)))
 
@@ -546,7 +608,10 @@ def run_b200(args):
                   "l2": f"{n_sets} rotating input/output sets ({n_sets * bytes_per_step / 1e6:.0f} MB"
                         f" > 3 x L2 {l2_bytes / 1e6:.0f} MB)",
                   "parallelism": f"dp{world}" if world > 1 else "single GPU"}
-        if isinstance(w, gen.DcnWorkload):
+        if isinstance(w, gen.DynWorkload):
+            config.update({"H": w.H, "W": w.W, "C": w.C, "G": w.G, "kernel": f"{w.K}x{w.K}",
+                           "softmax": bool(w.softmax_flag), "offsets": "none (ContMix core)"})
+        elif isinstance(w, gen.DcnWorkload):
             config.update({"H": w.H, "W": w.W, "C": w.C, "G": w.G, "kernel": f"{w.kh}x{w.kw}",
                            "stride": w.stride, "pad": w.pad, "dil": w.dil,
                            "softmax": bool(w.softmax_flag), "offset_sigma_px": w.offset_sigma})
@@ -574,7 +639,9 @@ def run_b200(args):
                          "kernel": kernel, "algorithmic_bytes_per_launch": bytes_per_step,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_src == "measured" else "fallback 6.65 TB/s"},
-            "on_chip": on_chip_roofline(w, ms_local / args.steps, sampler, device),
+            "on_chip": (fma_roofline(w, ms_local / args.steps, sampler, device)
+                        if isinstance(w, gen.DynWorkload)
+                        else on_chip_roofline(w, ms_local / args.steps, sampler, device)),
             "e2e": {"value": taps_total / (e2e_ms * 1e-3), "unit": "taps/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "steps": e2e_steps},
@@ -609,7 +676,7 @@ def run_reference(args):
     dt, taps = oracle_step(probe, seed=0, backward=backward)
     rate = taps / dt
     budget = 60.0 / max(1, args.steps + args.warmup)
-    if isinstance(w, gen.DcnWorkload):
+    if isinstance(w, (gen.DcnWorkload, gen.DynWorkload)):
         per_image = w.taps() / w.N
         n = max(1, min(w.N, int(budget * rate / per_image)))
         if budget * rate < per_image:     # less than one image: crop its rows
@@ -630,7 +697,7 @@ def run_reference(args):
         total_taps += taps
     value = total_taps / total_t
     sample = (f"each step: oracle on {step_w.name} with N={step_w.N}"
-              + (f", H={step_w.H}" if isinstance(step_w, gen.DcnWorkload) else
+              + (f", H={step_w.H}" if isinstance(step_w, (gen.DcnWorkload, gen.DynWorkload)) else
                  f", Lq={step_w.queries}")
               + f" ({step_w.taps()} taps), single thread, float64")
     return {

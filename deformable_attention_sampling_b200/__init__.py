@@ -10,6 +10,7 @@ binding: it marshals pointers, sizes and streams and runs nothing itself.
     out = dcnb.msda(value, shapes, starts, loc, attn)
     gx, goff, gmask = dcnb.dcn_grad(x, offset, mask, grad_out)
     gv, gloc, gattn = dcnb.msda_grad(value, shapes, starts, loc, attn, grad_out)
+    out = dcnb.dynconv(x, weights, K)        # ContMix core: per-pixel K x K kernels
 """
 from ._binding import (  # noqa: F401
     DCN_ERR_CUDA,
@@ -34,6 +35,8 @@ from ._binding import (  # noqa: F401
     dcn_status_string,
     dcn_version,
     dtype_code,
+    dynconv,
+    dynconv_forward,
     library,
     msda,
     msda_backward,

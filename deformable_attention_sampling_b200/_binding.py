@@ -34,6 +34,7 @@ SIGNATURES = {
     "dcn_backward_static_scratch": (_I, [_VP] * 7 + [_I] * 12 + [_VP]),
     "msda_backward_workspace_size": (_LL, [_I] * 5),
     "msda_backward": (_I, [_VP] * 10 + [_LL] + [_I] * 8 + [_VP]),
+    "dynconv_forward": (_I, [_VP] * 3 + [_I] * 8 + [_VP]),
     "dcn_output_size": (_I, [_I] * 5),
     "dcn_status_string": (ctypes.c_char_p, [_I]),
     "dcn_last_cuda_error": (_I, []),
@@ -160,6 +161,13 @@ def msda_backward(value, spatial_shapes, level_start, sampling_loc, attn_w, grad
                                  _ptr(workspace), workspace_bytes, N, S, Lq, M, D, L, K, dtype,
                                  _stream(stream)),
            "msda_backward")
+
+
+def dynconv_forward(x, weights, out, N, H, W, C, G, K, softmax_flag, dtype, stream=None):
+    """C dynconv_forward; raises DcnError on a non-OK status."""
+    _check(_load().dynconv_forward(_ptr(x), _ptr(weights), _ptr(out), N, H, W, C, G, K,
+                                   softmax_flag, dtype, _stream(stream)),
+           "dynconv_forward")
 
 
 def dcn_output_size(n_in, k, stride, pad, dil):
@@ -326,3 +334,24 @@ def msda_grad(value, spatial_shapes, level_start, sampling_loc, attn_w, grad_out
     msda_backward(value, spatial_shapes, level_start, sampling_loc, attn_w, grad_out, gv, gl, ga,
                   ws, ws_bytes, N, S, Lq, M, D, L, K, code, stream)
     return gv, gl, ga
+
+
+def dynconv(x, weights, K, softmax_flag=1, out=None, stream=None):
+    """dynconv_forward (the ContMix core) on torch CUDA tensors.
+
+    x [N, H, W, C], weights [N, H, W, G, K*K] (tap ky * K + kx), one dtype.
+    """
+    import torch
+    _require(x.dim() == 4 and weights.dim() == 5, "expected x [N,H,W,C], weights [N,H,W,G,K*K]")
+    N, H, W, C = x.shape
+    G = weights.shape[3]
+    _require(tuple(weights.shape) == (N, H, W, G, K * K), "weights has the wrong shape")
+    _require(weights.dtype == x.dtype, "mixed dtypes")
+    for t in (x, weights):
+        _require(t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(x)
+    _require(tuple(out.shape) == (N, H, W, C) and out.dtype == x.dtype and out.is_contiguous(),
+             "out has the wrong shape, dtype or layout")
+    dynconv_forward(x, weights, out, N, H, W, C, G, K, softmax_flag, dtype_code(x), stream)
+    return out

@@ -17,7 +17,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIB_DIR, "libdcn_b200.so")
 SOURCES = [os.path.join(CSRC, "dcn_abi.cu")]
-DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("common.cuh", "dcn_fwd.cuh", "msda_fwd.cuh", "dcn_bwd.cuh", "msda_bwd.cuh")]
+DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("common.cuh", "dcn_fwd.cuh", "msda_fwd.cuh", "dcn_bwd.cuh", "msda_bwd.cuh",
+                                                   "dynconv_fwd.cuh")]
 DEPENDS.append(os.path.join(INCLUDE, "dcn.h"))
 
 NVCC_FLAGS = [

@@ -13,6 +13,7 @@
 #include "dcn.h"
 #include "dcn_bwd.cuh"
 #include "dcn_fwd.cuh"
+#include "dynconv_fwd.cuh"
 #include "msda_bwd.cuh"
 #include "msda_fwd.cuh"
 
@@ -151,6 +152,26 @@ int launch(const void* fn, const Args& args, int num_blocks, int threads, int sm
     if (err != cudaSuccess) {
         g_last_cuda_error = (int)err;
         (void)cudaGetLastError();   // clear the launch error we just reported
+        return DCN_ERR_CUDA;
+    }
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return DCN_OK;
+}
+
+// One CTA per work unit (no persistent loop): the grid is the unit count.
+template <typename Args>
+int launch_grid(const void* fn, const Args& args, int num_blocks, int threads, int smem,
+                void* stream) {
+    if (wave_size(fn, threads, smem) <= 0) {   // sets the shared-memory attributes
+        g_last_cuda_error = (int)cudaGetLastError();
+        return DCN_ERR_CUDA;
+    }
+    void* params[] = {const_cast<Args*>(&args)};
+    const cudaError_t err = cudaLaunchKernel(fn, dim3(num_blocks), dim3(threads), params,
+                                             (size_t)smem, (cudaStream_t)stream);
+    if (err != cudaSuccess) {
+        g_last_cuda_error = (int)err;
+        (void)cudaGetLastError();
         return DCN_ERR_CUDA;
     }
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -706,6 +727,74 @@ int dcn_backward(const void* x, const void* offset, const void* mask, const void
     rc = launch(fn, b, a.num_tiles, 32 * warps, slice * warps, stream);
     if (rc != DCN_OK) return rc;
     return launch_round_dtype(dtype, acc, grad_x, acc_elems, stream);
+}
+
+int dynconv_forward(const void* x, const void* weights, void* out, int N, int H, int W, int C,
+                    int G, int K, int softmax_flag, int dtype, void* stream) {
+    const int es = elem_bytes(dtype);
+    if (es == 0 || N < 0 || H <= 0 || W <= 0 || C <= 0 || G <= 0 || C % G != 0 || K <= 0 ||
+        K % 2 != 1 || (softmax_flag != 0 && softmax_flag != 1))
+        return DCN_ERR_INVALID_ARG;
+    const int D = C / G;
+    if (K > dcnb::kDynMaxK || H > kMaxDim || W > kMaxDim || (D * es) % 32 != 0)
+        return DCN_ERR_UNSUPPORTED;
+    const long long pixels = (long long)N * H * W;
+    if ((long long)H * W * C * es > kInt31 || pixels * G > kInt31 ||
+        (long long)H * W * G * K * K > kInt31)
+        return DCN_ERR_UNSUPPORTED;
+    if (N == 0) return DCN_OK;
+    if (!x || !weights || !out) return DCN_ERR_INVALID_ARG;
+    if ((uintptr_t)x % 16 != 0 || (uintptr_t)out % 32 != 0 || (uintptr_t)weights % es != 0)
+        return DCN_ERR_MISALIGNED;
+    const long long xb = pixels * C * es;
+    if (overlaps(out, xb, x, xb) || overlaps(out, xb, weights, pixels * G * K * K * es))
+        return DCN_ERR_INVALID_ARG;
+
+    // tile rows: 8 on maps up to 64 rows (more CTAs), else 16
+    const int th = H <= 64 ? 8 : 16;
+    dcnb::DynArgs a;
+    a.x = x;
+    a.w = weights;
+    a.out = out;
+    a.H = H;
+    a.W = W;
+    a.C = C;
+    a.G = G;
+    a.D = D;
+    a.K = K;
+    a.th = th;
+    a.tiles_x = (W + dcnb::kDynTileW - 1) / dcnb::kDynTileW;
+    a.tiles_y = (H + th - 1) / th;
+    a.chunks = D * es / 32;
+    a.win_rows = th + K - 1;
+    a.row_bytes = dcnb::dyn_row_bytes(dcnb::kDynTileW + K - 1);
+    a.xs_bytes = a.win_rows * a.row_bytes;
+    a.ws_bytes = ((K * dcnb::dyn_wstride(th) * 4) + 15) & ~15;
+    const int raw_bytes =
+        2 * th * (dcnb::kDynTileW + 1) * dcnb::dyn_raw_words(K, es) * 4;   // two buffers
+    const int smem = a.xs_bytes + a.ws_bytes + raw_bytes + th * dcnb::kDynTileW * 4;
+    if (smem > kMaxBwdSmemBytes) return DCN_ERR_UNSUPPORTED;
+    const long long ctas = (long long)N * a.tiles_y * a.tiles_x * G * a.chunks;
+    if (ctas > kInt31) return DCN_ERR_UNSUPPORTED;
+
+    const void* fn = nullptr;
+    switch (dtype) {
+        case DCN_F32:
+            fn = softmax_flag ? (const void*)dcnb::dynconv_fwd_kernel<float, true>
+                              : (const void*)dcnb::dynconv_fwd_kernel<float, false>;
+            break;
+        case DCN_F16:
+            fn = softmax_flag ? (const void*)dcnb::dynconv_fwd_kernel<__half, true>
+                              : (const void*)dcnb::dynconv_fwd_kernel<__half, false>;
+            break;
+        case DCN_BF16:
+            fn = softmax_flag ? (const void*)dcnb::dynconv_fwd_kernel<__nv_bfloat16, true>
+                              : (const void*)dcnb::dynconv_fwd_kernel<__nv_bfloat16, false>;
+            break;
+        default: break;
+    }
+    if (!fn) return DCN_ERR_UNSUPPORTED;
+    return launch_grid(fn, a, (int)ctas, th * dcnb::kDynSegs, smem, stream);
 }
 
 long long msda_backward_workspace_size(int N, int S, int M, int D, int dtype) {

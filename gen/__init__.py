@@ -87,6 +87,36 @@ class DcnWorkload:
 
 
 @dataclass(frozen=True)
+class DynWorkload:
+    """Dynamic local aggregation (ContMix core): per-pixel K x K kernels."""
+    name: str
+    N: int
+    H: int
+    W: int
+    C: int
+    G: int
+    K: int
+    dtype: str = "f16"
+    softmax_flag: int = 1
+
+    @property
+    def D(self):
+        return self.C // self.G
+
+    def taps(self):
+        """weighted reads: one per (pixel, group, kernel tap)."""
+        return self.N * self.H * self.W * self.G * self.K * self.K
+
+    def pixels(self):
+        return self.N * self.H * self.W
+
+    def compulsory_bytes(self):
+        """x, weights and out, each read or written once."""
+        es = DTYPES[self.dtype].itemsize
+        return (2 * self.pixels() * self.C + self.taps()) * es
+
+
+@dataclass(frozen=True)
 class MsdaWorkload:
     name: str
     N: int
@@ -148,6 +178,10 @@ WORKLOADS = {w.name: w for w in [
     # DCNv4 fp16 at dense-prediction resolution with heavy-tailed offsets
     DcnWorkload("dcnv4_f16_2x200x320x64_g4", N=2, H=200, W=320, C=64, G=4, dtype="f16",
                 offset_sigma=8.0),
+    # ContMix core (dynamic K x K kernels, softmax) at the first-stage shape:
+    # the 7 x 7 and 13 x 13 kernel sizes of the OverLoCK networks
+    DynWorkload("contmix_f16_64x56x56x64_g4_k7", N=64, H=56, W=56, C=64, G=4, K=7),
+    DynWorkload("contmix_f16_64x56x56x64_g4_k13", N=64, H=56, W=56, C=64, G=4, K=13),
     # MSDeformAttn, four levels, encoder-style queries
     MsdaWorkload("msda_f32_2x4lvl_m8_d32_k4", N=2, M=8, D=32,
                  shapes=((100, 150), (50, 75), (25, 38), (13, 19)), K=4, dtype="f32"),
@@ -169,6 +203,15 @@ def dcn_inputs(w, seed=0):
     mask = rng.normal(0.0, 1.0, size=(w.N, w.Ho, w.Wo, w.G, w.K))
     return {"x": _round(x, w.dtype), "offset": _round(offset, w.dtype),
             "mask": _round(mask, w.dtype)}
+
+
+def dynconv_inputs(w, seed=0):
+    """x [N,H,W,C] ~ U[-1,1]; weights [N,H,W,G,K*K] ~ N(0, 1) (the numbers a
+    softmax turns into each location's kernel).  CPU tensors."""
+    rng = np.random.default_rng(seed)
+    x = rng.uniform(-1.0, 1.0, size=(w.N, w.H, w.W, w.C))
+    weights = rng.normal(0.0, 1.0, size=(w.N, w.H, w.W, w.G, w.K * w.K))
+    return {"x": _round(x, w.dtype), "weights": _round(weights, w.dtype)}
 
 
 def level_start_index(shapes):

@@ -257,6 +257,35 @@ DCN_API int msda_backward(const void* value, const int64_t* spatial_shapes,
                   void* workspace, long long workspace_bytes, int N, int S, int Lq, int M,
                   int D, int L, int K, int dtype, void* stream);
 
+/*
+ * dynconv_forward - dynamic local aggregation (the ContMix core), forward.
+ *
+ * Defined by the "OverLoCK" note, "ContMix: Put the Whole Image into the
+ * Kernel", steps 4-5: a softmax turns each location's K*K numbers into its own
+ * K x K kernel per channel group, which is applied to the zero-padded K x K
+ * neighbourhood of that group's channels (taps row-major, as the note's unfold
+ * with padding K / 2 orders them).  For every pixel (y, x), group g < G and
+ * channel c < D = C / G:
+ *
+ *   out[n][y][x][g*D + c] = sum_{ky, kx < K} A[ky*K + kx] * x[n][y + ky - K/2][x + kx - K/2][g*D + c]
+ *     A = softmax over t of weights[n][y][x][g][t]   (softmax_flag = 1)
+ *     A = weights[n][y][x][g][.] as given             (softmax_flag = 0)
+ *   with x = 0 outside the map.  It is dcn_forward with every offset zero,
+ *   stride 1, pad K / 2, and the tap order ky * K + kx.
+ *
+ * Layouts: x [N][H][W][C], weights [N][H][W][G][K*K], out [N][H][W][C].
+ * Limits: K odd, K <= 31; one group's channels a multiple of 32 bytes
+ * (D * element size % 32 == 0: 16 f16 / bf16 or 8 f32 channels per 32 bytes);
+ * H, W <= 65536; one image of x below 2^31 bytes (DCN_ERR_UNSUPPORTED
+ * otherwise).  N = 0 launches nothing.
+ * Errors: DCN_ERR_INVALID_ARG for a bad dimension, an even K, C % G != 0,
+ * softmax_flag not 0/1, an unknown dtype, a null pointer (N > 0) or out
+ * overlapping an input; DCN_ERR_MISALIGNED unless x is 16-byte aligned, out
+ * 32-byte aligned and weights aligned to the element size.
+ */
+DCN_API int dynconv_forward(const void* x, const void* weights, void* out, int N, int H,
+                 int W, int C, int G, int K, int softmax_flag, int dtype, void* stream);
+
 /* Output size of the deformable window: (in + 2 pad - dil (k - 1) - 1) / stride + 1,
  * or a value <= 0 when the window does not fit. */
 DCN_API int dcn_output_size(int in, int k, int stride, int pad, int dil);

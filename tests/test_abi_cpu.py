@@ -231,3 +231,32 @@ def test_msda_backward_validation(lib, change, status):
     before = dcnb.dcn_launch_count()
     assert call_msda_bwd(lib, **change) == status
     assert dcnb.dcn_launch_count() == before
+
+
+def call_dyn(lib, **kw):
+    args = dict(x=X, w=OFF, out=OUT, N=2, H=8, W=8, C=32, G=2, K=7, softmax_flag=1, dtype=F16,
+                stream=None)
+    args.update(kw)
+    a = args
+    return lib.dynconv_forward(a["x"], a["w"], a["out"], a["N"], a["H"], a["W"], a["C"], a["G"],
+                               a["K"], a["softmax_flag"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(dtype=5), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(K=4), dcnb.DCN_ERR_INVALID_ARG),              # even window
+    (dict(K=0), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(C=33), dcnb.DCN_ERR_INVALID_ARG),             # C % G != 0
+    (dict(softmax_flag=2), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(K=33), dcnb.DCN_ERR_UNSUPPORTED),
+    (dict(C=16, G=2), dcnb.DCN_ERR_UNSUPPORTED),        # D * 2 bytes = 16, not a multiple of 32
+    (dict(x=None), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(out=X), dcnb.DCN_ERR_INVALID_ARG),            # out aliases x
+    (dict(x=X + 8), dcnb.DCN_ERR_MISALIGNED),
+    (dict(out=OUT + 16), dcnb.DCN_ERR_MISALIGNED),
+    (dict(N=0), dcnb.DCN_OK),
+])
+def test_dynconv_validation(lib, change, status):
+    before = dcnb.dcn_launch_count()
+    assert call_dyn(lib, **change) == status
+    assert dcnb.dcn_launch_count() == before

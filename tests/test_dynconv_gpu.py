@@ -1,0 +1,97 @@
+"""GPU parity of dynconv_forward (the ContMix core) against the float64
+oracle (tests/parity.py tolerances), through the C interface: the full-size
+workloads in the benchmark's launch configuration (checked on sampled batch
+items: an output depends on its own image only), then small shapes across
+tile edges, window sizes, group widths, dtypes and both weight modes."""
+import numpy as np
+import pytest
+import torch
+
+import deformable_attention_sampling_b200 as dcnb
+import gen
+import oracle
+from tests.parity import compare
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def run(inp, w):
+    out = dcnb.dynconv(inp["x"].to(DEV), inp["weights"].to(DEV), w.K, w.softmax_flag)
+    torch.cuda.synchronize()
+    return out
+
+
+def ref(inp, w, n=None):
+    sel = (lambda t: t[n:n + 1]) if n is not None else (lambda t: t)
+    return oracle.dynconv_forward_ref(sel(inp["x"]), sel(inp["weights"]), w.K, w.softmax_flag)
+
+
+DYN_WORKLOADS = [n for n, w in gen.WORKLOADS.items() if isinstance(w, gen.DynWorkload)]
+
+
+@pytest.mark.parametrize("name", DYN_WORKLOADS)
+def test_dynconv_workload_full_size(name):
+    w = gen.WORKLOADS[name]
+    inp = gen.dynconv_inputs(w, seed=0)
+    out = run(inp, w)
+    for n in sorted({0, w.N // 2, w.N - 1}):
+        compare(out[n:n + 1], ref(inp, w, n), f"{name} image {n}")
+
+
+SMALL = [
+    # N, H, W, C, G, K, dtype, softmax
+    (1, 1, 1, 16, 1, 1, "f16", 1),
+    (2, 5, 7, 32, 2, 3, "f16", 1),
+    (1, 9, 33, 64, 4, 5, "bf16", 1),       # a second, ragged column tile
+    (1, 67, 40, 16, 1, 7, "f16", 1),       # more than 64 rows: 16-row tiles
+    (2, 13, 70, 32, 1, 13, "f16", 0),      # D = 32: two 32-byte channel chunks
+    (1, 6, 6, 16, 2, 13, "f32", 1),        # D = 8 fp32; window wider than the map
+    (1, 20, 24, 48, 3, 17, "bf16", 1),     # more than 16 taps per kernel row
+    (1, 5, 5, 16, 1, 31, "f16", 1),        # the largest window on a tiny map
+    (3, 8, 12, 24, 3, 9, "f32", 0),        # D = 8 fp32, weights used as given
+    (1, 31, 29, 64, 4, 7, "f32", 1),       # D = 16 fp32: two chunks
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[f"case{i}" for i in range(len(SMALL))])
+def test_dynconv_small_shapes(case):
+    N, H, W, C, G, K, dt, sm = case
+    w = gen.DynWorkload("small", N=N, H=H, W=W, C=C, G=G, K=K, dtype=dt, softmax_flag=sm)
+    inp = gen.dynconv_inputs(w, seed=3)
+    compare(run(inp, w), ref(inp, w), str(case))
+
+
+def test_dynconv_large_logits_and_one_launch():
+    """Logits far from 0 (the max subtraction keeps exp finite), one launch."""
+    w = gen.DynWorkload("big", N=2, H=10, W=11, C=32, G=2, K=5, dtype="f32")
+    inp = gen.dynconv_inputs(w, seed=4)
+    inp["weights"] = inp["weights"] * 40.0 + 60.0
+    before = dcnb.dcn_launch_count()
+    out = run(inp, w)
+    assert dcnb.dcn_launch_count() - before == 1
+    compare(out, ref(inp, w), "large logits")
+
+
+def test_dynconv_x_on_a_16_byte_boundary_and_errors():
+    w = gen.DynWorkload("mis", N=1, H=6, W=9, C=16, G=1, K=3, dtype="f16")
+    inp = gen.dynconv_inputs(w, seed=5)
+    buf = torch.empty(inp["x"].numel() + 8, dtype=torch.float16, device=DEV)
+    x = buf[8:].view(inp["x"].shape)          # 16 bytes past a 32-byte boundary
+    x.copy_(inp["x"].to(DEV))
+    out = dcnb.dynconv(x, inp["weights"].to(DEV), w.K)
+    torch.cuda.synchronize()
+    compare(out, ref(inp, w), "x at 16 bytes")
+    bad = torch.empty(out.numel() + 8, dtype=torch.float16, device=DEV)[8:].view(out.shape)
+    with pytest.raises(dcnb.DcnError) as e:
+        dcnb.dynconv(x, inp["weights"].to(DEV), w.K, out=bad)
+    assert e.value.status == dcnb.DCN_ERR_MISALIGNED
+
+
+def test_dynconv_empty_batch():
+    x = torch.empty((0, 4, 4, 16), dtype=torch.float16, device=DEV)
+    wt = torch.empty((0, 4, 4, 1, 9), dtype=torch.float16, device=DEV)
+    before = dcnb.dcn_launch_count()
+    out = dcnb.dynconv(x, wt, 3)
+    assert dcnb.dcn_launch_count() == before and out.shape == x.shape
+    assert np.prod(out.shape) == 0
