@@ -744,7 +744,7 @@ int dynconv_forward(const void* x, const void* weights, void* out, int N, int H,
         return DCN_ERR_UNSUPPORTED;
     if (N == 0) return DCN_OK;
     if (!x || !weights || !out) return DCN_ERR_INVALID_ARG;
-    if ((uintptr_t)x % 16 != 0 || (uintptr_t)out % 32 != 0 || (uintptr_t)weights % es != 0)
+    if ((uintptr_t)x % 16 != 0 || (uintptr_t)out % 32 != 0 || (uintptr_t)weights % 16 != 0)
         return DCN_ERR_MISALIGNED;
     const long long xb = pixels * C * es;
     if (overlaps(out, xb, x, xb) || overlaps(out, xb, weights, pixels * G * K * K * es))
@@ -770,9 +770,8 @@ int dynconv_forward(const void* x, const void* weights, void* out, int N, int H,
     a.row_bytes = dcnb::dyn_row_bytes(dcnb::kDynTileW + K - 1);
     a.xs_bytes = a.win_rows * a.row_bytes;
     a.ws_bytes = ((K * dcnb::dyn_wstride(th) * 4) + 15) & ~15;
-    const int raw_bytes =
-        2 * th * (dcnb::kDynTileW + 1) * dcnb::dyn_raw_words(K, es) * 4;   // two buffers
-    const int smem = a.xs_bytes + a.ws_bytes + raw_bytes + th * dcnb::kDynTileW * 4;
+    const int raw_bytes = 2 * th * dcnb::kDynTileW * dcnb::dyn_slot_bytes(K, es);   // two buffers
+    const int smem = a.xs_bytes + a.ws_bytes + raw_bytes;
     if (smem > kMaxBwdSmemBytes) return DCN_ERR_UNSUPPORTED;
     const long long ctas = (long long)N * a.tiles_y * a.tiles_x * G * a.chunks;
     if (ctas > kInt31) return DCN_ERR_UNSUPPORTED;

@@ -20,14 +20,16 @@
 //             the 32-byte loads of a warp (threads 4 columns apart) spread over
 //             all banks.
 //   weights = one kernel row (ky) at a time: the K numbers of every location
-//             are copied by lane groups with coalesced loads into a
-//             double-buffered raw shared buffer (the next row is fetched while
-//             the current one is used), then the thread that owns a location
-//             turns them into float32 weights in its own slots [kx][row][col]
-//             (row stride 33: conflict-free).  With the softmax the maximum of
-//             each location's K*K numbers comes from a pre-pass, each weight is
-//             exp2((z - max) log2 e), computed once, the owner sums them in
-//             registers and divides its outputs by the sum at the end.
+//             are copied with 16-byte cp.async blocks (from the block that holds
+//             the first number, the last copy clipped to the row's end) into a
+//             double-buffered raw shared buffer, the next row in flight while
+//             the current one is used; the thread that owns a location reads
+//             them at any alignment and writes float32 weights into its own
+//             slots [kx][row][col] (row stride 33: conflict-free).  The softmax
+//             runs online per location: a running maximum keeps exp finite,
+//             each weight is exp2((z - max) log2 e), computed once, and the
+//             running sum and the owner's accumulators are rescaled when the
+//             maximum grows; the output is divided by the sum at the end.
 // Per kernel row the thread slides along x: each window pixel it loads (two
 // 16-byte shared loads, widened once) is multiplied into the up to four
 // outputs whose taps cover it, with packed FFMA2 into float32 accumulators.
@@ -68,39 +70,27 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t 
                  "r"(src_bytes) : "memory");
 }
 
-constexpr int kDynStageUnroll = 8;   // loads in flight per lane while staging weights
-
-// Words per location in the raw weight buffer: the K numbers of one kernel row
-// (16-bit or 32-bit), rounded up to an odd count so that the locations a warp
-// reads at once fall in different banks.
-__host__ __device__ inline int dyn_raw_words(int K, int es) {
-    const int w = (K * es + 3) / 4;
-    return w | 1;
-}
+// Bytes of one location's slot in the raw weight buffer: the K numbers of a
+// kernel row start anywhere within their first 16-byte block, so the slot
+// holds ceil((K * es + 15) / 16) whole blocks.
+__host__ __device__ inline int dyn_slot_bytes(int K, int es) { return ((K * es + 15 + 15) / 16) * 16; }
 
 template <typename T, bool SOFTMAX>
 __global__ void __launch_bounds__(256) dynconv_fwd_kernel(const DynArgs a) {
     constexpr int CPT = 32 / (int)sizeof(T);
     constexpr int es = (int)sizeof(T);
-    constexpr int U = kDynStageUnroll;
     constexpr float kLog2e = 1.4426950408889634f;
     extern __shared__ __align__(16) unsigned char smem[];
     const int TH = a.th;
     const int NP = TH * kDynTileW;                  // locations of the tile
     const int K = a.K, KK = K * K, r = K >> 1;
-    const int RW = dyn_raw_words(K, es);            // raw words per location
-    const int RP = kDynTileW + 1;                   // locations per raw / ws row (padded)
+    const int SB = dyn_slot_bytes(K, es);
     unsigned char* xs = smem;
     float* ws = reinterpret_cast<float*>(smem + a.xs_bytes);
-    uint32_t* raw = reinterpret_cast<uint32_t*>(smem + a.xs_bytes + a.ws_bytes);
-    const int raw_words = TH * RP * RW;             // one buffer
-    float* s_max = reinterpret_cast<float*>(raw + 2 * raw_words);
+    unsigned char* raw = smem + a.xs_bytes + a.ws_bytes;   // two buffers of NP slots
 
     const int tid = threadIdx.x;
     const int nthreads = blockDim.x;
-    const int lane = tid & 31;
-    const int warp = tid >> 5;
-    const int nwarps = nthreads >> 5;
 
     // tile coordinates: blockIdx.x = (((n * tiles_y + ty) * tiles_x + tx) * G + g) * chunks + q
     int b = blockIdx.x;
@@ -137,56 +127,28 @@ __global__ void __launch_bounds__(256) dynconv_fwd_kernel(const DynArgs a) {
     const int w_col = a.G * KK;
     const int w_row = a.W * w_col;
     auto in_map = [&](int row, int col) { return y0 + row < a.H && x0 + col < a.W; };
+    // slot of location (row, col): ordered [col % 4][row][col / 4], so that the
+    // owners of one column offset read consecutive slots
+    auto slot = [&](int row, int col) { return ((col & 3) * TH + row) * kDynSegs + (col >> 2); };
 
-    // ---- softmax: maximum of each location's K*K numbers (a warp per location) ----
-    if constexpr (SOFTMAX) {
-        for (int pix0 = warp * 4; pix0 < NP; pix0 += nwarps * 4) {
-            float m[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int pix = pix0 + u;
-                const int row = pix / kDynTileW, col = pix - row * kDynTileW;
-                m[u] = -INFINITY;
-                if (pix < NP && in_map(row, col)) {
-                    const T* wp = wt + row * w_row + col * w_col;
-                    for (int t = lane; t < KK; t += 32) m[u] = fmaxf(m[u], Elem<T>::one(wp + t));
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    m[u] = fmaxf(m[u], __shfl_xor_sync(0xffffffffu, m[u], o));
-                if (lane == 0 && pix0 + u < NP) s_max[pix0 + u] = m[u];
-            }
-        }
-    }
-
-    // Copy kernel row ky of every location into raw buffer `buf` (lanes over
-    // the K numbers of a location, 16 or 32 lanes per location, U locations in
-    // flight per lane).  Locations outside the map copy nothing.
-    const int lpp = K <= 16 ? 16 : 32;
-    const int ppw = 32 / lpp;
-    const int sub = lane / lpp, kx_l = lane - sub * lpp;
+    // Copy kernel row ky of every location of the tile into raw buffer `buf`:
+    // whole 16-byte blocks from the block holding the row's first number,
+    // each copy clipped to the row's last byte (nothing past it is read).
     auto copy_row = [&](int ky, int buf) {
-        T* dst = reinterpret_cast<T*>(raw + buf * raw_words);
-        for (int base = warp * ppw * U; base < NP; base += nwarps * ppw * U) {
-            T v[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int pix = base + u * ppw + sub;
-                const int row = pix / kDynTileW, col = pix - row * kDynTileW;
-                if (pix < NP && kx_l < K && in_map(row, col))
-                    v[u] = wt[row * w_row + col * w_col + ky * K + kx_l];
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int pix = base + u * ppw + sub;
-                const int row = pix / kDynTileW, col = pix - row * kDynTileW;
-                if (pix < NP && kx_l < K && in_map(row, col))
-                    dst[(row * RP + col) * RW * (4 / es) + kx_l] = v[u];
+        unsigned char* dst0 = raw + buf * NP * SB;
+        for (int loc = tid; loc < NP; loc += nthreads) {
+            const int row = loc / kDynTileW, col = loc - row * kDynTileW;
+            if (!in_map(row, col)) continue;
+            const char* first = reinterpret_cast<const char*>(wt + row * w_row + col * w_col + ky * K);
+            const char* last = first + K * es;
+            const char* blk = reinterpret_cast<const char*>((uintptr_t)first & ~(uintptr_t)15);
+            unsigned char* dst = dst0 + slot(row, col) * SB;
+            for (; blk < last; blk += 16, dst += 16) {
+                const long long left = last - blk;
+                cp_async16(dst, blk, left >= 16 ? 16u : (uint32_t)left);
             }
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
     // ---- this thread's outputs: 4 columns of one row ----
@@ -198,51 +160,62 @@ __global__ void __launch_bounds__(256) dynconv_fwd_kernel(const DynArgs a) {
     for (int p = 0; p < kDynP; ++p)
 #pragma unroll
         for (int i = 0; i < CPT; ++i) acc[p][i] = 0.f;
-    float mloc[kDynP], ssum[kDynP];
+    float mrun[kDynP], ssum[kDynP];
     bool mine[kDynP];
-
-    const int wstride = dyn_wstride(TH);
-    copy_row(0, 0);
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    __syncthreads();
+    int skew[kDynP];    // byte offset of the row's first number within its block
 #pragma unroll
     for (int p = 0; p < kDynP; ++p) {
         mine[p] = in_map(row, col0 + p);
-        mloc[p] = SOFTMAX && mine[p] ? s_max[row * kDynTileW + col0 + p] * kLog2e : 0.f;
+        mrun[p] = -INFINITY;
         ssum[p] = 0.f;
+        skew[p] = (int)((uintptr_t)(wt + row * w_row + (col0 + p) * w_col) & 15);
     }
+    const int wstride = dyn_wstride(TH);
+    float* wk = ws + row * (kDynTileW + 1) + col0;
 
+    copy_row(0, 0);
     for (int ky = 0; ky < K; ++ky) {
-        if (ky > 0) __syncthreads();   // raw row ky complete; raw row ky - 1 consumed
-        // this thread's weights of kernel row ky: exp (softmax) once per tap,
-        // into its own slots of ws (read back only by this thread)
-        {
-            const T* src = reinterpret_cast<const T*>(raw + (ky & 1) * raw_words);
-            float* wk = ws + row * RP + col0;
+        if (ky + 1 < K) {
+            if (ky > 0) __syncthreads();      // raw buffer (ky + 1) & 1 is no longer read
+            copy_row(ky + 1, (ky + 1) & 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");   // window and row ky landed
+        } else {
+            asm volatile("cp.async.wait_all;" ::: "memory");
+        }
+        __syncthreads();
+
+        // this thread's weights of kernel row ky, into its own slots of ws
 #pragma unroll
-            for (int p = 0; p < kDynP; ++p) {
-                const T* rp = src + (row * RP + col0 + p) * RW * (4 / es);
+        for (int p = 0; p < kDynP; ++p) {
+            if (!mine[p]) {
+                for (int kx = 0; kx < K; ++kx) wk[kx * wstride + p] = 0.f;
+                continue;
+            }
+            const int sk = (skew[p] + ky * K * es) & 15;
+            const T* zr = reinterpret_cast<const T*>(raw + (ky & 1) * NP * SB +
+                                                     slot(row, col0 + p) * SB + sk);
+            if constexpr (SOFTMAX) {
+                float m = mrun[p];
+                for (int kx = 0; kx < K; ++kx) m = fmaxf(m, Elem<T>::one(zr + kx));
+                const float sc = exp2f((mrun[p] - m) * kLog2e);   // 0 on the first row
+                mrun[p] = m;
+                const float ml = m * kLog2e;
+                float srow = 0.f;
                 for (int kx = 0; kx < K; ++kx) {
-                    float e = 0.f;
-                    if (mine[p]) {
-                        const float z = Elem<T>::one(rp + kx);
-                        if constexpr (SOFTMAX) {
-                            e = exp2f(fmaf(z, kLog2e, -mloc[p]));
-                            ssum[p] += e;
-                        } else {
-                            e = z;
-                        }
-                    }
+                    const float e = exp2f(fmaf(Elem<T>::one(zr + kx), kLog2e, -ml));
+                    srow += e;
                     wk[kx * wstride + p] = e;
                 }
+                ssum[p] = fmaf(ssum[p], sc, srow);
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) acc[p][i] *= sc;
+            } else {
+                for (int kx = 0; kx < K; ++kx) wk[kx * wstride + p] = Elem<T>::one(zr + kx);
             }
         }
-        // prefetch kernel row ky + 1 into the other buffer while computing
-        if (ky + 1 < K) copy_row(ky + 1, (ky + 1) & 1);
 
         // slide along the window row (row + ky) over columns col0 .. col0 + K + P - 2
         const unsigned char* xrow = xs + (row + ky) * a.row_bytes;
-        const float* wk = ws + row * RP + col0;
         for (int j = 0; j < K + kDynP - 1; ++j) {
             const unsigned char* px = xrow + dyn_pixel_byte(col0 + j);
             uint32_t wv[8];

@@ -280,8 +280,8 @@ DCN_API int msda_backward(const void* value, const int64_t* spatial_shapes,
  * otherwise).  N = 0 launches nothing.
  * Errors: DCN_ERR_INVALID_ARG for a bad dimension, an even K, C % G != 0,
  * softmax_flag not 0/1, an unknown dtype, a null pointer (N > 0) or out
- * overlapping an input; DCN_ERR_MISALIGNED unless x is 16-byte aligned, out
- * 32-byte aligned and weights aligned to the element size.
+ * overlapping an input; DCN_ERR_MISALIGNED unless x and weights are 16-byte
+ * aligned and out is 32-byte aligned.
  */
 DCN_API int dynconv_forward(const void* x, const void* weights, void* out, int N, int H,
                  int W, int C, int G, int K, int softmax_flag, int dtype, void* stream);
