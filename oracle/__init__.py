@@ -190,3 +190,46 @@ def dynconv_forward_ref(x, weights, K, softmax_flag=1, groups=None):
     if rc != 0:
         raise ValueError("oracle_dynconv_forward rejected its arguments")
     return out
+
+
+def msda_locations_ref(spatial_shapes, reference, offsets, valid_ratios=None):
+    """float64 sampling locations of the reference-point variants.
+
+    reference [N, Lq, 2] points or [N, Lq, 4] boxes (cx, cy, w, h) in
+    valid-image coordinates; offsets [N, Lq, M, L, K, 2]; valid_ratios
+    [N, L, 2] as (W_valid / W, H_valid / H), or None for all 1.  Applies
+    scalar.sampling_location_ref element by element -> loc [N, Lq, M, L, K, 2].
+    """
+    ref = _as_f64(reference)
+    off = _as_f64(offsets)
+    shapes = np.asarray(spatial_shapes, dtype=np.int64)
+    N, Lq, M, L, K, _ = off.shape
+    vr = np.ones((N, L, 2)) if valid_ratios is None else _as_f64(valid_ratios)
+    loc = np.empty_like(off)
+    for n in range(N):
+        for q in range(Lq):
+            for m in range(M):
+                for l in range(L):
+                    wh = (float(shapes[l][1]), float(shapes[l][0]))
+                    for k in range(K):
+                        loc[n, q, m, l, k] = scalar.sampling_location_ref(
+                            ref[n, q], off[n, q, m, l, k], wh, K, vr[n, l])
+    return loc
+
+
+def mask_value_ref(value, mask):
+    """value [N, S, M, D] with every row whose mask [N, S] is set replaced by 0
+    (Deformable DETR: the attention module zeroes projected values at masked
+    positions)."""
+    v = _as_f64(value).copy()
+    m = np.asarray(mask).astype(bool)
+    v[m] = 0.0
+    return v
+
+
+def msda_points_ref(value, spatial_shapes, level_start, reference, offsets, attn,
+                    valid_ratios=None):
+    """float64 MSDA core fed from references: the locations of
+    msda_locations_ref, then msda_forward_ref."""
+    loc = msda_locations_ref(spatial_shapes, reference, offsets, valid_ratios)
+    return msda_forward_ref(value, spatial_shapes, level_start, loc, attn)

@@ -102,6 +102,27 @@ def sampling_location(reference, offset, shape_wh):
             reference[1] + offset[1] / shape_wh[1]]
 
 
+def sampling_location_ref(reference, offset, shape_wh, points, valid_ratio=(1.0, 1.0)):
+    """Point or box reference to a normalised location in a padded level.
+
+    Deformable DETR, "A reference links resolutions without equating their
+    pixels" and helper 1: the reference is in valid-image coordinates and is
+    scaled by the level's valid ratio r = (W_valid / W, H_valid / H); a 2-D
+    point adds offset / (W, H); a 4-D box (cx, cy, w, h) adds
+    (offset / points) * (w, h) * r / 2 instead.  No clamping.
+    `shape_wh` is the padded level size (width, height).
+    """
+    out = []
+    for axis in range(2):
+        centre = reference[axis] * valid_ratio[axis]
+        if len(reference) == 4:
+            shift = offset[axis] / points * reference[axis + 2] * valid_ratio[axis] / 2.0
+        else:
+            shift = offset[axis] / shape_wh[axis]
+        out.append(centre + shift)
+    return out
+
+
 def out_size(n_in, k, stride, pad, dil):
     return (n_in + 2 * pad - dil * (k - 1) - 1) // stride + 1
 
