@@ -418,7 +418,55 @@ class DynRunner:
         return self.w.compulsory_bytes()
 
 
+class MsdaPointsRunner:
+    """One step = one msda_forward_points call (locations formed in-kernel
+    from box / point references and valid ratios)."""
+    kernel = "msda_fwd_kernel (reference-point variant)"
+
+    def __init__(self, w, seed, device):
+        import deformable_attention_sampling_b200 as dcnb
+        self.dcnb = dcnb
+        self.w = w
+        self.host = {k: v for k, v in gen.msda_ref_inputs(w, seed=seed).items() if k != "mask"}
+        self.device = device
+        self.code = gen.DTYPE_CODES[w.dtype]
+        self.lib = dcnb.library()
+
+    def alloc_set(self):
+        d = {k: v.to(self.device) for k, v in self.host.items()}
+        d["out"] = torch.empty((self.w.N, self.w.queries, self.w.M * self.w.D),
+                               dtype=self.host["value"].dtype, device=self.device)
+        return d
+
+    def launcher(self, s, stream):
+        w, lib = self.w, self.lib
+        args = (s["value"].data_ptr(), s["spatial_shapes"].data_ptr(),
+                s["level_start"].data_ptr(), s["reference"].data_ptr(), w.ref_dim,
+                s["valid_ratios"].data_ptr(), s["offsets"].data_ptr(), s["attn"].data_ptr(),
+                s["out"].data_ptr(), w.N, w.queries, w.M, w.D, w.L, w.K, self.code, stream)
+
+        def go():
+            st = lib.msda_forward_points(*args)
+            if st != 0:
+                raise self.dcnb.DcnError(st, "msda_forward_points")
+        return go
+
+    def inputs_of(self, s):
+        return [(s[k], self.host[k]) for k in ("value", "spatial_shapes", "level_start",
+                                               "reference", "valid_ratios", "offsets", "attn")]
+
+    def outputs_of(self, s):
+        return [s["out"]]
+
+    def bytes_per_step(self):
+        return self.w.compulsory_bytes()
+
+
 def make_runner(w, seed, device, backward=False):
+    if isinstance(w, gen.MsdaWorkload) and w.ref_dim:
+        if backward:
+            raise SystemExit("--pass backward is not offered for the reference-point variants")
+        return MsdaPointsRunner(w, seed, device)
     if isinstance(w, gen.DynWorkload):
         if backward:
             raise SystemExit("--pass backward is not offered for the ContMix workloads")
@@ -440,6 +488,11 @@ def oracle_step(w, seed, backward=False):
         t = time.perf_counter()
         oracle.dcn_backward_ref(inp["x"], inp["offset"], inp["mask"], go, w.kh, w.kw, w.stride,
                                 w.pad, w.dil, w.softmax_flag)
+    elif isinstance(w, gen.MsdaWorkload) and w.ref_dim:
+        inp = gen.msda_ref_inputs(w, seed=seed)
+        t = time.perf_counter()
+        oracle.msda_points_ref(inp["value"], inp["spatial_shapes"], inp["level_start"],
+                               inp["reference"], inp["offsets"], inp["attn"], inp["valid_ratios"])
     elif backward:
         inp = gen.msda_inputs(w, seed=seed)
         go = gen.grad_out((w.N, w.queries, w.M * w.D), w.dtype, seed)
@@ -618,6 +671,9 @@ def run_b200(args):
         else:
             config.update({"M": w.M, "D": w.D, "levels": [list(s) for s in w.shapes],
                            "K": w.K, "Lq": w.queries})
+            if w.ref_dim:
+                config.update({"reference": "box (cx, cy, w, h)" if w.ref_dim == 4 else "point",
+                               "valid_ratios": "U[0.75, 1] per (image, level, axis)"})
         result = {
             "metric": metric_name(w, backward),
             "value": value,

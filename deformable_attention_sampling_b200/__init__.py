@@ -42,5 +42,9 @@ from ._binding import (  # noqa: F401
     msda_backward,
     msda_backward_workspace_size,
     msda_forward,
+    msda_forward_points,
+    msda_mask_value,
+    msda_points,
+    mask_value,
     msda_grad,
 )

@@ -29,6 +29,8 @@ _LL = ctypes.c_longlong
 SIGNATURES = {
     "dcn_forward": (_I, [_VP, _VP, _VP, _VP] + [_I] * 12 + [_VP]),
     "msda_forward": (_I, [_VP] * 6 + [_I] * 7 + [_VP]),
+    "msda_forward_points": (_I, [_VP] * 4 + [_I] + [_VP] * 4 + [_I] * 7 + [_VP]),
+    "msda_mask_value": (_I, [_VP] * 3 + [_I] * 5 + [_VP]),
     "dcn_backward_workspace_size": (_LL, [_I] * 5),
     "dcn_backward": (_I, [_VP] * 8 + [_LL] + [_I] * 12 + [_VP]),
     "dcn_backward_static_scratch": (_I, [_VP] * 7 + [_I] * 12 + [_VP]),
@@ -168,6 +170,23 @@ def dynconv_forward(x, weights, out, N, H, W, C, G, K, softmax_flag, dtype, stre
     _check(_load().dynconv_forward(_ptr(x), _ptr(weights), _ptr(out), N, H, W, C, G, K,
                                    softmax_flag, dtype, _stream(stream)),
            "dynconv_forward")
+
+
+def msda_forward_points(value, spatial_shapes, level_start, reference, ref_dim, valid_ratios,
+                        offsets, attn_w, out, N, Lq, M, D, L, K, dtype, stream=None):
+    """C msda_forward_points; raises DcnError on a non-OK status."""
+    _check(_load().msda_forward_points(_ptr(value), _ptr(spatial_shapes), _ptr(level_start),
+                                       _ptr(reference), ref_dim, _ptr(valid_ratios),
+                                       _ptr(offsets), _ptr(attn_w), _ptr(out), N, Lq, M, D, L,
+                                       K, dtype, _stream(stream)),
+           "msda_forward_points")
+
+
+def msda_mask_value(value, mask, out, N, S, M, D, dtype, stream=None):
+    """C msda_mask_value; raises DcnError on a non-OK status."""
+    _check(_load().msda_mask_value(_ptr(value), _ptr(mask), _ptr(out), N, S, M, D, dtype,
+                                   _stream(stream)),
+           "msda_mask_value")
 
 
 def dcn_output_size(n_in, k, stride, pad, dil):
@@ -354,4 +373,41 @@ def dynconv(x, weights, K, softmax_flag=1, out=None, stream=None):
     _require(tuple(out.shape) == (N, H, W, C) and out.dtype == x.dtype and out.is_contiguous(),
              "out has the wrong shape, dtype or layout")
     dynconv_forward(x, weights, out, N, H, W, C, G, K, softmax_flag, dtype_code(x), stream)
+    return out
+
+
+def msda_points(value, spatial_shapes, level_start, reference, offsets, attn_w,
+                valid_ratios=None, out=None, stream=None):
+    """msda_forward_points on torch CUDA tensors: reference [N, Lq, 2 or 4],
+    offsets [N, Lq, M, L, K, 2], valid_ratios [N, L, 2] or None."""
+    import torch
+    N, S, M, D = value.shape
+    _, Lq, _, L, K = attn_w.shape
+    ref_dim = reference.shape[-1]
+    _require(tuple(reference.shape) == (N, Lq, ref_dim) and ref_dim in (2, 4),
+             "reference must be [N, Lq, 2] or [N, Lq, 4]")
+    _require(tuple(offsets.shape) == (N, Lq, M, L, K, 2), "offsets has the wrong shape")
+    _require(valid_ratios is None or tuple(valid_ratios.shape) == (N, L, 2),
+             "valid_ratios must be [N, L, 2]")
+    for t in (value, reference, offsets, attn_w) + ((valid_ratios,) if valid_ratios is not None else ()):
+        _require(t.is_cuda and t.is_contiguous() and t.dtype == value.dtype,
+                 "tensors must be contiguous CUDA tensors of one dtype")
+    if out is None:
+        out = torch.empty((N, Lq, M * D), dtype=value.dtype, device=value.device)
+    msda_forward_points(value, spatial_shapes, level_start, reference, ref_dim, valid_ratios,
+                        offsets, attn_w, out, N, Lq, M, D, L, K, dtype_code(value), stream)
+    return out
+
+
+def mask_value(value, mask, out=None, stream=None):
+    """msda_mask_value on torch CUDA tensors (mask [N, S] bool or uint8);
+    out=value masks in place."""
+    import torch
+    N, S, M, D = value.shape
+    _require(tuple(mask.shape) == (N, S), "mask must be [N, S]")
+    m = mask.to(torch.uint8) if mask.dtype != torch.uint8 else mask
+    _require(m.is_cuda and m.is_contiguous() and value.is_contiguous(), "contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(value)
+    msda_mask_value(value, m, out, N, S, M, D, dtype_code(value), stream)
     return out

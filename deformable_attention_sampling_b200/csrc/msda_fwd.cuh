@@ -41,7 +41,7 @@ struct MsdaArgs {
     const void* value;
     const int64_t* shapes;       // [L][2] (H_l, W_l), device
     const int64_t* level_start;  // [L], device
-    const void* loc;
+    const void* loc;             // locations, or offsets for the reference variants
     const void* attn;
     void* out;
     int Lq, M, D, L, K;
@@ -51,6 +51,8 @@ struct MsdaArgs {
     int num_runs;                // ceil(total_items / run_items)
     int stage_elems;             // staged weights per warp (run_items * L * K); 0 = unstaged
     FastDiv div_M, div_Lq, div_tpi;
+    const void* ref;             // reference variants: [N][Lq][2 or 4] in valid-image units
+    const void* vr;              // [N][L][2] valid ratios (W_valid / W, H_valid / H) or null
 };
 
 // Integer cell and fraction of the normalised coordinate u on a level of
@@ -80,13 +82,34 @@ struct MsdaTap {
     float w[4];
 };
 
+// Cell and fraction of a pixel-space coordinate x (already u W - 1/2),
+// formed in double precision by the caller: a few float32 roundings of a
+// position near 150 px would already move samples by ~1e-5 px.
+__device__ __forceinline__ float pixel_coord(double x, int* cell) {
+    double fx = floor(x);
+    const float a = fminf(fmaxf((float)(x - fx), 0.f), 1.f);   // NaN: far outside, a = 0
+    fx = fmin(fmax(fx, -4194304.0), 4194304.0);                // +-2^22
+    *cell = (int)fx;
+    return a;
+}
+
+__device__ __forceinline__ MsdaTap msda_corners(const int (*lvl)[3], long long pix_bytes, int l,
+                                                int x0, float ax, int y0, float ay, float A);
+
 __device__ __forceinline__ MsdaTap msda_tap(const int (*lvl)[3], long long pix_bytes, int l,
                                             float u, float v, float A) {
-    MsdaTap t;
     const int Hl = lvl[l][0], Wl = lvl[l][1];
     int x0, y0;
     const float ax = level_coord(u, (float)Wl, &x0);
     const float ay = level_coord(v, (float)Hl, &y0);
+    return msda_corners(lvl, pix_bytes, l, x0, ax, y0, ay, A);
+}
+
+// The four corners of cell (x0, y0) with fractions (ax, ay) on level l.
+__device__ __forceinline__ MsdaTap msda_corners(const int (*lvl)[3], long long pix_bytes, int l,
+                                                int x0, float ax, int y0, float ay, float A) {
+    MsdaTap t;
+    const int Hl = lvl[l][0], Wl = lvl[l][1];
     const int x1 = x0 + 1, y1 = y0 + 1;
     const bool vx0 = (unsigned)x0 < (unsigned)Wl, vx1 = (unsigned)x1 < (unsigned)Wl;
     const bool vy0 = (unsigned)y0 < (unsigned)Hl, vy1 = (unsigned)y1 < (unsigned)Hl;
@@ -135,7 +158,14 @@ __device__ __forceinline__ void msda_warp_stage(T* dst, const T* src, int elems,
     }
 }
 
-template <typename T, int VB>
+// REF = 0: sampling_loc holds the normalised locations.  REF = 2 / 4: it holds
+// the offsets of the reference-point variants ("Deformable DETR", "A reference
+// links resolutions without equating their pixels" and helper 1), and the
+// pixel position is formed here from the point (cx, cy) or box (cx, cy, w, h)
+// reference of the query and the level's valid ratio r:
+//   point: x = (cx r) W + dx - 1/2                  (s = cx r + dx / W)
+//   box:   x = ((cx + dx w / (2K)) r) W - 1/2       (s = cx r + dx / K * w * r / 2)
+template <typename T, int VB, int REF = 0>
 __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArgs a) {
     constexpr int CPT = VB / (int)sizeof(T);
     constexpr int NW = VB >= 4 ? VB / 4 : 1;
@@ -199,6 +229,20 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArg
         const char* vb = static_cast<const char*>(a.value) +
                          ((long long)n * s_S * a.M + h) * a.D * (int)sizeof(T) +
                          (long long)chunk * CPT * (int)sizeof(T);
+        // reference variants: the query's reference, the batch item's ratios
+        float rcx = 0.f, rcy = 0.f, rw = 0.f, rh = 0.f;
+        const T* vrp = nullptr;
+        if constexpr (REF != 0) {
+            const T* rp = static_cast<const T*>(a.ref) + (long long)nq * REF;
+            rcx = Elem<T>::one(rp);
+            rcy = Elem<T>::one(rp + 1);
+            if constexpr (REF == 4) {   // box size (w, h)
+                rw = Elem<T>::one(rp + 2);
+                rh = Elem<T>::one(rp + 3);
+            }
+            if (a.vr) vrp = static_cast<const T*>(a.vr) + (long long)n * L * 2;
+        }
+        float rx = 1.f, ry = 1.f;   // valid ratios of the current level
 
         float acc[CPT];
 #pragma unroll
@@ -211,7 +255,29 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArg
         auto geometry = [&]() {
             float u, vv;
             load_pair<T>(locp + 2 * nt, u, vv);
-            const MsdaTap t = msda_tap(s_lvl, pix_bytes, nl, u, vv, Elem<T>::one(wp + nt));
+            MsdaTap t;
+            if constexpr (REF == 0) {
+                t = msda_tap(s_lvl, pix_bytes, nl, u, vv, Elem<T>::one(wp + nt));
+            } else {
+                if (vrp && nt == nl * K) {    // first tap of a level
+                    rx = Elem<T>::one(vrp + 2 * nl);
+                    ry = Elem<T>::one(vrp + 2 * nl + 1);
+                }
+                const double Wl = (double)s_lvl[nl][1], Hl = (double)s_lvl[nl][0];
+                double x, y;
+                if constexpr (REF == 2) {
+                    x = fma((double)rcx * rx, Wl, (double)u) - 0.5;
+                    y = fma((double)rcy * ry, Hl, (double)vv) - 0.5;
+                } else {
+                    const double half_k = 0.5 / (double)K;
+                    x = fma((double)u * half_k, (double)rw, (double)rcx) * rx * Wl - 0.5;
+                    y = fma((double)vv * half_k, (double)rh, (double)rcy) * ry * Hl - 0.5;
+                }
+                int x0, y0;
+                const float ax = pixel_coord(x, &x0);
+                const float ay = pixel_coord(y, &y0);
+                t = msda_corners(s_lvl, pix_bytes, nl, x0, ax, y0, ay, Elem<T>::one(wp + nt));
+            }
             ++nt;
             if (nt == (nl + 1) * K) ++nl;
             return t;
@@ -247,6 +313,44 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArg
         char* ob = static_cast<char*>(a.out) +
                    ((long long)nq * a.M * a.D + h * a.D + chunk * CPT) * (int)sizeof(T);
         store_vec<VB>(ob, o);
+    }
+}
+
+}  // namespace dcnb
+
+namespace dcnb {
+
+// value rows whose mask byte is set become 0 ("Deformable DETR": the attention
+// module zeroes projected values at masked positions); out may be value.
+struct MaskArgs {
+    const void* value;
+    const unsigned char* mask;   // [N][S]
+    void* out;
+    long long rows;              // N * S
+    int row_bytes;               // M * D * element size
+    int vec16;                   // 1: rows, value and out are 16-byte aligned
+};
+
+__global__ void __launch_bounds__(256) msda_mask_value_kernel(const MaskArgs m) {
+    const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long nthreads = (long long)gridDim.x * blockDim.x;
+    const char* src = static_cast<const char*>(m.value);
+    char* dst = static_cast<char*>(m.out);
+    if (m.vec16) {
+        const int per_row = m.row_bytes >> 4;
+        const long long total = m.rows * per_row;
+        for (long long i = tid; i < total; i += nthreads) {
+            const long long row = i / per_row;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (!m.mask[row]) v = reinterpret_cast<const uint4*>(src)[i];
+            reinterpret_cast<uint4*>(dst)[i] = v;
+        }
+    } else {
+        const long long total = m.rows * m.row_bytes;
+        for (long long i = tid; i < total; i += nthreads) {
+            const long long row = i / m.row_bytes;
+            dst[i] = m.mask[row] ? 0 : src[i];
+        }
     }
 }
 

@@ -127,6 +127,7 @@ class MsdaWorkload:
     Lq: int = 0               # 0: one query per pixel of all levels (encoder style)
     dtype: str = "f32"
     offset_sigma: float = 2.0  # std of the pixel offsets at each level
+    ref_dim: int = 0          # 2 / 4: reference points / boxes with valid ratios
 
     @property
     def L(self):
@@ -147,12 +148,15 @@ class MsdaWorkload:
         return self.N * self.queries
 
     def compulsory_bytes(self):
+        """value, locations (or offsets), weights and out once; the reference
+        variants add the references and the valid ratios."""
         es = DTYPES[self.dtype].itemsize
         value = self.N * self.S * self.M * self.D
         loc = self.taps() * 2
         w = self.taps()
         out = self.N * self.queries * self.M * self.D
-        return (value + loc + w + out) * es
+        refs = self.N * self.queries * self.ref_dim + (self.N * self.L * 2 if self.ref_dim else 0)
+        return (value + loc + w + out + refs) * es
 
     def backward_bytes(self):
         """value, locations, weights and grad_out read once; grad_value,
@@ -185,6 +189,11 @@ WORKLOADS = {w.name: w for w in [
     # MSDeformAttn, four levels, encoder-style queries
     MsdaWorkload("msda_f32_2x4lvl_m8_d32_k4", N=2, M=8, D=32,
                  shapes=((100, 150), (50, 75), (25, 38), (13, 19)), K=4, dtype="f32"),
+    # the same levels as a decoder with 4-D box references, valid ratios and
+    # 300 object queries per image
+    MsdaWorkload("msda_f32_2x4lvl_m8_d32_k4_box300", N=2, M=8, D=32,
+                 shapes=((100, 150), (50, 75), (25, 38), (13, 19)), K=4, Lq=300, dtype="f32",
+                 ref_dim=4),
 ]}
 
 HEADLINE = "dcnv4_f16_64x56x56x64_g4"
@@ -254,6 +263,51 @@ def grad_out(shape, dtype, seed=0):
     forward inputs of the same seed are unchanged."""
     rng = np.random.default_rng([seed, 0x6772])
     return _round(rng.normal(0.0, 1.0, size=tuple(shape)), dtype)
+
+
+def msda_ref_inputs(w, seed=0):
+    """Inputs of the reference-point variants (ref_dim 2 or 4): value as
+    msda_inputs; valid ratios ~U[0.75, 1] per (n, level, axis) (right / bottom
+    padding); points ~U[0,1]^2 in valid-image units, or boxes with centre
+    ~U[0,1]^2 and size ~U[0.05, 0.3]; offsets ~N(0, sigma) (pixels for points,
+    units of box size * K / 2 for boxes, so sigma / K box half-sizes); weights
+    normalised jointly over (l, k); a padding mask [N, S] of the value rows
+    beyond each level's valid extent."""
+    rng = np.random.default_rng(seed)
+    Lq = w.queries
+    value = rng.uniform(-1.0, 1.0, size=(w.N, w.S, w.M, w.D))
+    vr = rng.uniform(0.75, 1.0, size=(w.N, w.L, 2))
+    if w.ref_dim == 4:
+        ref = np.concatenate([rng.uniform(0.0, 1.0, size=(w.N, Lq, 2)),
+                              rng.uniform(0.05, 0.3, size=(w.N, Lq, 2))], axis=-1)
+        sigma = 1.0
+    else:
+        ref = rng.uniform(0.0, 1.0, size=(w.N, Lq, 2))
+        sigma = w.offset_sigma
+    off = rng.normal(0.0, sigma, size=(w.N, Lq, w.M, w.L, w.K, 2))
+    logits = rng.normal(0.0, 1.0, size=(w.N, Lq, w.M, w.L, w.K))
+    flat = logits.reshape(w.N, Lq, w.M, w.L * w.K)
+    e = np.exp(flat - flat.max(axis=-1, keepdims=True))
+    attn = (e / e.sum(axis=-1, keepdims=True)).reshape(logits.shape)
+    mask = np.zeros((w.N, w.S), dtype=bool)
+    starts = level_start_index(w.shapes)
+    for n in range(w.N):
+        for l, (h, wd) in enumerate(w.shapes):
+            hv = int(np.ceil(vr[n, l, 1] * h))
+            wv = int(np.ceil(vr[n, l, 0] * wd))
+            m = np.ones((h, wd), dtype=bool)
+            m[:hv, :wv] = False
+            mask[n, starts[l]:starts[l] + h * wd] = m.reshape(-1)
+    return {
+        "value": _round(value, w.dtype),
+        "spatial_shapes": torch.tensor(w.shapes, dtype=torch.int64),
+        "level_start": torch.tensor(starts, dtype=torch.int64),
+        "reference": _round(ref, w.dtype),
+        "valid_ratios": _round(vr, w.dtype),
+        "offsets": _round(off, w.dtype),
+        "attn": _round(attn, w.dtype),
+        "mask": torch.from_numpy(mask),
+    }
 
 
 def scaled(w, **changes):

@@ -131,6 +131,48 @@ DCN_API int msda_forward(const void* value, const int64_t* spatial_shapes,
                  int L, int K, int dtype, void* stream);
 
 /*
+ * msda_forward_points - msda_forward fed from reference points or boxes.
+ *
+ * Defined by "Deformable DETR: Learn Where to Read", "A reference links
+ * resolutions without equating their pixels" and helper 1: a query's
+ * reference is in valid-image coordinates; level l's valid ratio r =
+ * (W_valid / W_l, H_valid / H_l) scales it into the level's padded frame, and
+ *   point reference (cx, cy):        s = (cx, cy) * r + offset / (W_l, H_l)
+ *   box reference (cx, cy, w, h):    s = (cx, cy) * r + offset / K * (w, h) * r / 2
+ * (componentwise, no clamping); then exactly msda_forward with location s.
+ * The locations are formed in the kernel and never stored.
+ *
+ * Arguments: as msda_forward, with
+ *   reference     [N][Lq][ref_dim]   ref_dim = 2 (point) or 4 (box), dtype
+ *   valid_ratios  [N][L][2]          (x, y) ratios in dtype, or NULL for all 1
+ *   offsets       [N][Lq][M][L][K][2] in place of sampling_loc
+ * Padding masks are not applied here: zero the masked value rows first
+ * (msda_mask_value), as the module does before the sampling core.
+ * Errors: as msda_forward; DCN_ERR_INVALID_ARG also for ref_dim not 2 / 4 or
+ * a NULL reference; DCN_ERR_MISALIGNED for a reference or ratio pointer not
+ * aligned to the element size.
+ */
+DCN_API int msda_forward_points(const void* value, const int64_t* spatial_shapes,
+                 const int64_t* level_start, const void* reference, int ref_dim,
+                 const void* valid_ratios, const void* offsets, const void* attn_w, void* out,
+                 int N, int Lq, int M, int D, int L, int K, int dtype, void* stream);
+
+/*
+ * msda_mask_value - zero the value rows of padded positions.
+ *
+ * "Deformable DETR", "A reference links resolutions ...": the attention module
+ * zeroes projected values at masked positions, so that a read near a
+ * valid-image edge mixes valid features with zeros.  For every n < N, s < S:
+ *   out[n][s][.][.] = mask[n][s] ? 0 : value[n][s][.][.]
+ * value / out [N][S][M][D] in dtype, mask [N][S] bytes (non-zero = masked).
+ * out may be value itself (in place); otherwise it must not overlap it.
+ * Errors: DCN_ERR_INVALID_ARG for a bad dimension, dtype, NULL pointer (N > 0)
+ * or overlap; DCN_ERR_MISALIGNED for value / out not aligned to the element size.
+ */
+DCN_API int msda_mask_value(const void* value, const unsigned char* mask, void* out, int N,
+                 int S, int M, int D, int dtype, void* stream);
+
+/*
  * dcn_backward_workspace_size - bytes of scratch that dcn_backward needs.
  *
  * grad_x is a scatter (every tap adds to four pixels), accumulated in float32:
