@@ -233,3 +233,29 @@ def msda_points_ref(value, spatial_shapes, level_start, reference, offsets, attn
     msda_locations_ref, then msda_forward_ref."""
     loc = msda_locations_ref(spatial_shapes, reference, offsets, valid_ratios)
     return msda_forward_ref(value, spatial_shapes, level_start, loc, attn)
+
+
+def dcnv4_front_end_ref(x, w_om, b_om, kh, kw, pad, dil, groups):
+    """float64 DCNv4 module core with its merged offset / mask linear.
+
+    "DCNv4" note, "1. Remove Softmax": one linear layer produces every
+    location's G*K offset pairs and G*K modulation scalars from the same
+    features, which then drive the sampling core (no softmax).  Here
+    om = x @ w_om^T + b_om per pixel (a library matmul in float64) with
+    w_om [G*K*3, C]; its first G*K*2 outputs are the offsets in [G][K][2]
+    order, the last G*K the masks in [G][K] order; stride 1, so the linear is
+    applied at every output pixel.  Returns (out, offset, mask).
+    """
+    x = _as_f64(x)
+    w = _as_f64(w_om)
+    N, H, W, C = x.shape
+    G = groups
+    K = kh * kw
+    om = x.reshape(-1, C) @ w.T
+    if b_om is not None:
+        om = om + _as_f64(b_om)[None, :]
+    offset = om[:, :G * K * 2].reshape(N, H, W, G, K, 2)
+    mask = om[:, G * K * 2:].reshape(N, H, W, G, K)
+    out = dcn_forward_ref(x, offset, mask, kh, kw, stride=1, pad=pad, dil=dil, softmax_flag=0,
+                          groups=G)
+    return out, offset, mask
