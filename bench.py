@@ -462,7 +462,52 @@ class MsdaPointsRunner:
         return self.w.compulsory_bytes()
 
 
+class FusedRunner:
+    """One step = one dcnv4_fused_forward call (merged offset / mask linear on
+    the tensor cores feeding the sampler; offsets never leave the SM)."""
+    kernel = "dcn_fwd_kernel (fused front end)"
+
+    def __init__(self, w, seed, device):
+        import deformable_attention_sampling_b200 as dcnb
+        self.dcnb = dcnb
+        self.w = w
+        self.host = gen.front_end_inputs(w, seed=seed)
+        self.device = device
+        self.code = gen.DTYPE_CODES[w.dtype]
+        self.lib = dcnb.library()
+
+    def alloc_set(self):
+        d = {k: v.to(self.device) for k, v in self.host.items()}
+        d["out"] = torch.empty_like(d["x"])
+        return d
+
+    def launcher(self, s, stream):
+        w, lib = self.w, self.lib
+        args = (s["x"].data_ptr(), s["w_om"].data_ptr(), s["b_om"].data_ptr(),
+                s["out"].data_ptr(), w.N, w.H, w.W, w.C, w.G, w.kh, w.kw, w.pad, w.dil,
+                self.code, stream)
+
+        def go():
+            st = lib.dcnv4_fused_forward(*args)
+            if st != 0:
+                raise self.dcnb.DcnError(st, "dcnv4_fused_forward")
+        return go
+
+    def inputs_of(self, s):
+        return [(s[k], self.host[k]) for k in ("x", "w_om", "b_om")]
+
+    def outputs_of(self, s):
+        return [s["out"]]
+
+    def bytes_per_step(self):
+        return self.w.compulsory_bytes()
+
+
 def make_runner(w, seed, device, backward=False):
+    if isinstance(w, gen.FusedWorkload):
+        if backward:
+            raise SystemExit("--pass backward is not offered for the fused front end")
+        return FusedRunner(w, seed, device)
     if isinstance(w, gen.MsdaWorkload) and w.ref_dim:
         if backward:
             raise SystemExit("--pass backward is not offered for the reference-point variants")
@@ -499,6 +544,11 @@ def oracle_step(w, seed, backward=False):
         t = time.perf_counter()
         oracle.msda_backward_ref(inp["value"], inp["spatial_shapes"], inp["level_start"],
                                  inp["loc"], inp["attn"], go)
+    elif isinstance(w, gen.FusedWorkload):
+        inp = gen.front_end_inputs(w, seed=seed)
+        t = time.perf_counter()
+        oracle.dcnv4_front_end_ref(inp["x"], inp["w_om"], inp["b_om"], w.kh, w.kw, w.pad, w.dil,
+                                   w.G)
     elif isinstance(w, gen.DynWorkload):
         inp = gen.dynconv_inputs(w, seed=seed)
         t = time.perf_counter()
@@ -519,7 +569,7 @@ def oracle_step(w, seed, backward=False):
 def sample_of(w, n_images):
     """A bounded sample of workload w with the same per-tap work: fewer batch
     items (DCN) or fewer queries (MSDA)."""
-    if isinstance(w, (gen.DcnWorkload, gen.DynWorkload)):
+    if isinstance(w, (gen.DcnWorkload, gen.DynWorkload, gen.FusedWorkload)):
         return gen.scaled(w, N=max(1, min(w.N, n_images)))
     return gen.scaled(w, N=1, Lq=max(1, min(w.queries, n_images * 64)))
 
@@ -661,7 +711,11 @@ def run_b200(args):
                   "l2": f"{n_sets} rotating input/output sets ({n_sets * bytes_per_step / 1e6:.0f} MB"
                         f" > 3 x L2 {l2_bytes / 1e6:.0f} MB)",
                   "parallelism": f"dp{world}" if world > 1 else "single GPU"}
-        if isinstance(w, gen.DynWorkload):
+        if isinstance(w, gen.FusedWorkload):
+            config.update({"H": w.H, "W": w.W, "C": w.C, "G": w.G, "kernel": f"{w.kh}x{w.kw}",
+                           "front_end": f"merged linear {w.C} -> {w.J} on the tensor cores",
+                           "offset_sigma_px": w.offset_sigma})
+        elif isinstance(w, gen.DynWorkload):
             config.update({"H": w.H, "W": w.W, "C": w.C, "G": w.G, "kernel": f"{w.K}x{w.K}",
                            "softmax": bool(w.softmax_flag), "offsets": "none (ContMix core)"})
         elif isinstance(w, gen.DcnWorkload):
@@ -732,7 +786,7 @@ def run_reference(args):
     dt, taps = oracle_step(probe, seed=0, backward=backward)
     rate = taps / dt
     budget = 60.0 / max(1, args.steps + args.warmup)
-    if isinstance(w, (gen.DcnWorkload, gen.DynWorkload)):
+    if isinstance(w, (gen.DcnWorkload, gen.DynWorkload, gen.FusedWorkload)):
         per_image = w.taps() / w.N
         n = max(1, min(w.N, int(budget * rate / per_image)))
         if budget * rate < per_image:     # less than one image: crop its rows
@@ -753,7 +807,8 @@ def run_reference(args):
         total_taps += taps
     value = total_taps / total_t
     sample = (f"each step: oracle on {step_w.name} with N={step_w.N}"
-              + (f", H={step_w.H}" if isinstance(step_w, (gen.DcnWorkload, gen.DynWorkload)) else
+              + (f", H={step_w.H}" if isinstance(step_w, (gen.DcnWorkload, gen.DynWorkload,
+                                                             gen.FusedWorkload)) else
                  f", Lq={step_w.queries}")
               + f" ({step_w.taps()} taps), single thread, float64")
     return {

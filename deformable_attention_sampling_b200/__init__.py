@@ -32,6 +32,8 @@ from ._binding import (  # noqa: F401
     dcn_last_cuda_error,
     dcn_launch_count,
     dcn_output_size,
+    dcnv4_fused,
+    dcnv4_fused_forward,
     dcn_status_string,
     dcn_version,
     dtype_code,

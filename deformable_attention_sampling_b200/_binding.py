@@ -37,6 +37,7 @@ SIGNATURES = {
     "msda_backward_workspace_size": (_LL, [_I] * 5),
     "msda_backward": (_I, [_VP] * 10 + [_LL] + [_I] * 8 + [_VP]),
     "dynconv_forward": (_I, [_VP] * 3 + [_I] * 8 + [_VP]),
+    "dcnv4_fused_forward": (_I, [_VP] * 4 + [_I] * 10 + [_VP]),
     "dcn_output_size": (_I, [_I] * 5),
     "dcn_status_string": (ctypes.c_char_p, [_I]),
     "dcn_last_cuda_error": (_I, []),
@@ -187,6 +188,14 @@ def msda_mask_value(value, mask, out, N, S, M, D, dtype, stream=None):
     _check(_load().msda_mask_value(_ptr(value), _ptr(mask), _ptr(out), N, S, M, D, dtype,
                                    _stream(stream)),
            "msda_mask_value")
+
+
+def dcnv4_fused_forward(x, w_om, b_om, out, N, H, W, C, G, kh, kw, pad, dil, dtype,
+                        stream=None):
+    """C dcnv4_fused_forward; raises DcnError on a non-OK status."""
+    _check(_load().dcnv4_fused_forward(_ptr(x), _ptr(w_om), _ptr(b_om), _ptr(out), N, H, W, C,
+                                       G, kh, kw, pad, dil, dtype, _stream(stream)),
+           "dcnv4_fused_forward")
 
 
 def dcn_output_size(n_in, k, stride, pad, dil):
@@ -410,4 +419,22 @@ def mask_value(value, mask, out=None, stream=None):
     if out is None:
         out = torch.empty_like(value)
     msda_mask_value(value, m, out, N, S, M, D, dtype_code(value), stream)
+    return out
+
+
+def dcnv4_fused(x, w_om, b_om=None, groups=4, kh=3, kw=3, pad=1, dil=1, out=None, stream=None):
+    """dcnv4_fused_forward on torch CUDA tensors: x [N, H, W, C], w_om
+    [G*kh*kw*3, C], b_om [G*kh*kw*3] or None."""
+    import torch
+    N, H, W, C = x.shape
+    J = groups * kh * kw * 3
+    _require(tuple(w_om.shape) == (J, C), "w_om must be [G*K*3, C]")
+    _require(b_om is None or tuple(b_om.shape) == (J,), "b_om must be [G*K*3]")
+    for t in (x, w_om) + ((b_om,) if b_om is not None else ()):
+        _require(t.is_cuda and t.is_contiguous() and t.dtype == x.dtype,
+                 "tensors must be contiguous CUDA tensors of one dtype")
+    if out is None:
+        out = torch.empty_like(x)
+    dcnv4_fused_forward(x, w_om, b_om, out, N, H, W, C, groups, kh, kw, pad, dil, dtype_code(x),
+                        stream)
     return out

@@ -33,6 +33,8 @@
 // The binding limit is the SM's L1 data path for scattered 32-byte gathers.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace dcnb {
@@ -67,7 +69,117 @@ struct DcnArgs {
     uint32_t pix_bytes;       // C * sizeof(T): byte stride between neighbouring pixels
     uint32_t row_bytes;       // W * C * sizeof(T)
     long long img_bytes;      // H * W * C * sizeof(T)
+    // fused front end only: the merged offset / mask linear
+    const void* w_om;         // [J][C], J = G * K * 3 (offsets in [G][K][2] order, then masks)
+    const void* b_om;         // [J] or null
+    int J;
 };
+
+// ---------------------------------------------- fused DCNv4 front end ----
+//
+// "DCNv4" note, "1. Remove Softmax": one linear layer gives every location its
+// G*K offset pairs and G*K modulation scalars.  In the fused kernel each warp
+// computes them for its run's pixels on the tensor cores (mma.sync m16n8k16,
+// 16-bit inputs, float32 accumulation: a 16-pixel x 8-output tile per
+// instruction) straight into its shared slice, in float32, so the offsets and
+// masks never travel through HBM and are never rounded to 16 bits.
+
+template <typename T>
+__device__ __forceinline__ void mma_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1);
+
+template <>
+__device__ __forceinline__ void mma_16816<__half>(float* c, const uint32_t* a, uint32_t b0,
+                                                  uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <>
+__device__ __forceinline__ void mma_16816<__nv_bfloat16>(float* c, const uint32_t* a, uint32_t b0,
+                                                         uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <>
+__device__ __forceinline__ void mma_16816<float>(float*, const uint32_t*, uint32_t, uint32_t) {}
+
+// Row stride (elements) of the staged weight matrix: C plus 8, so that the
+// eight rows a B fragment reads start in different banks.
+__host__ __device__ inline int fused_w_stride(int C) { return C + 8; }
+
+// om[pixel][j] = sum_c W[j][c] x[pixel][c] + b[j] for the npix pixels of one
+// run (row `xrow`, first pixel pix0), written to s_off[pixel * 2GK + j]
+// (j < 2GK) and s_mask[pixel * GK + j - 2GK].  Ws: staged W (rows padded to
+// a multiple of 16 with zeros), bs: bias.  All 32 lanes take part.
+constexpr int kFusedMaxKSteps = 8;   // C <= 128: the A fragments of a run stay in registers
+
+template <typename T>
+__device__ __forceinline__ void fused_front_end(const T* xrow, int pix0, int npix, int C, int J,
+                                                int GK, const T* Ws, const float* bs,
+                                                float* s_off, float* s_mask, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+    const int WS = fused_w_stride(C);
+    const int G2K = 2 * GK;
+    const int KS = C >> 4;
+    for (int m0 = 0; m0 < npix; m0 += 16) {
+        const int r0 = m0 + gid, r1 = m0 + gid + 8;           // this lane's two pixel rows
+        // the run's A fragments for every k-step, loaded once
+        uint32_t afr[kFusedMaxKSteps][4];
+        {
+            const T* x0 = xrow + (long long)(pix0 + r0) * C + 2 * tig;
+            const T* x1 = xrow + (long long)(pix0 + r1) * C + 2 * tig;
+#pragma unroll
+            for (int ks = 0; ks < kFusedMaxKSteps; ++ks) {
+                afr[ks][0] = afr[ks][1] = afr[ks][2] = afr[ks][3] = 0u;
+                if (ks < KS) {
+                    if (r0 < npix) {
+                        afr[ks][0] = *reinterpret_cast<const uint32_t*>(x0 + ks * 16);
+                        afr[ks][2] = *reinterpret_cast<const uint32_t*>(x0 + ks * 16 + 8);
+                    }
+                    if (r1 < npix) {
+                        afr[ks][1] = *reinterpret_cast<const uint32_t*>(x1 + ks * 16);
+                        afr[ks][3] = *reinterpret_cast<const uint32_t*>(x1 + ks * 16 + 8);
+                    }
+                }
+            }
+        }
+        // two 8-output tiles per step: independent accumulator chains
+        for (int n0 = 0; n0 < J; n0 += 16) {
+            float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            const T* w0 = Ws + (n0 + gid) * WS + 2 * tig;
+            const T* w1 = w0 + 8 * WS;
+#pragma unroll
+            for (int ks = 0; ks < kFusedMaxKSteps; ++ks) {
+                if (ks < KS) {
+                    mma_16816<T>(c[0], afr[ks], *reinterpret_cast<const uint32_t*>(w0 + ks * 16),
+                                 *reinterpret_cast<const uint32_t*>(w0 + ks * 16 + 8));
+                    mma_16816<T>(c[1], afr[ks], *reinterpret_cast<const uint32_t*>(w1 + ks * 16),
+                                 *reinterpret_cast<const uint32_t*>(w1 + ks * 16 + 8));
+                }
+            }
+            // epilogue: c[t][0..1] row r0, c[t][2..3] row r1, outputs j and j + 1
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int j = n0 + 8 * t + 2 * tig;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = e < 2 ? r0 : r1;
+                    const int jj = j + (e & 1);
+                    if (r < npix && jj < J) {
+                        const float v = c[t][e] + bs[jj];
+                        if (jj < G2K) s_off[r * G2K + jj] = v;
+                        else s_mask[r * GK + (jj - G2K)] = v;
+                    }
+                }
+            }
+        }
+    }
+}
 
 // Copy `elems` elements of T from global `src` to shared `dst` with the lanes
 // of one warp (widest access the addresses and size allow; streaming loads).
@@ -193,11 +305,15 @@ __device__ __forceinline__ TapGeom tap_geometry(const DcnArgs& a, int bxk, int b
 // KF > 0: a fixed KF x KF window, whose taps are fully unrolled (tap indices,
 // kernel offsets and shared-memory addresses fold into constants; measured
 // 10% faster for 3 x 3).  KF = 0: any window, taps in a rolled loop.
-template <typename T, int VB, bool SOFTMAX, int KF = 0>
+// FUSED: offsets and masks come from the merged linear of the DCNv4 front end
+// (fused_front_end, float32 in shared memory) instead of global tensors;
+// stride 1, runs aligned to whole pixels (checked on the host).
+template <typename T, int VB, bool SOFTMAX, int KF = 0, bool FUSED = false>
 __global__ void __launch_bounds__(kDcnMaxThreads, 1) dcn_fwd_kernel(const DcnArgs a) {
     constexpr int UNROLL = KF ? KF * KF : 1;
     constexpr int CPT = VB / (int)sizeof(T);
     constexpr int NW = VB >= 4 ? VB / 4 : 1;
+    using OT = typename std::conditional<FUSED, float, T>::type;   // staged offset / mask type
     extern __shared__ __align__(16) unsigned char smem[];
 
     const int kh = KF ? KF : a.kh;
@@ -205,12 +321,34 @@ __global__ void __launch_bounds__(kDcnMaxThreads, 1) dcn_fwd_kernel(const DcnArg
     const int K = kh * kw;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const bool staged = a.stage_elems > 0;
+    const bool staged = FUSED || a.stage_elems > 0;
+    // fused: the staged weight matrix and bias come first
+    unsigned char* wsm = smem;
+    int front = 0;
+    if constexpr (FUSED) {
+        const int rows = (a.J + 15) & ~15;
+        front = ((rows * fused_w_stride(a.C) * (int)sizeof(T) + 15) & ~15) + ((a.J * 4 + 15) & ~15);
+    }
     // this warp's slice of shared memory: offsets, then masks
-    const int off_slice = ((2 * a.stage_elems * (int)sizeof(T)) + 15) & ~15;
-    const int slice = off_slice + ((a.stage_elems * (int)sizeof(T) + 15) & ~15);
-    T* s_off = reinterpret_cast<T*>(smem + warp * slice);
-    T* s_mask = reinterpret_cast<T*>(smem + warp * slice + off_slice);
+    const int off_slice = ((2 * a.stage_elems * (int)sizeof(OT)) + 15) & ~15;
+    const int slice = off_slice + ((a.stage_elems * (int)sizeof(OT) + 15) & ~15);
+    OT* s_off = reinterpret_cast<OT*>(smem + front + warp * slice);
+    OT* s_mask = reinterpret_cast<OT*>(smem + front + warp * slice + off_slice);
+    if constexpr (FUSED) {
+        // stage W (rows padded to a multiple of 16 with zeros) and the bias
+        const int rows = (a.J + 15) & ~15;
+        const int WS = fused_w_stride(a.C);
+        T* Ws = reinterpret_cast<T*>(wsm);
+        const T* wg = static_cast<const T*>(a.w_om);
+        for (int e = threadIdx.x; e < rows * a.C; e += blockDim.x) {
+            const int j = e / a.C, c = e - j * a.C;
+            Ws[j * WS + c] = j < a.J ? wg[e] : Elem<T>::from(0.f);
+        }
+        float* bs = reinterpret_cast<float*>(wsm + ((rows * WS * (int)sizeof(T) + 15) & ~15));
+        for (int j = threadIdx.x; j < a.J; j += blockDim.x)
+            bs[j] = a.b_om ? Elem<T>::one(static_cast<const T*>(a.b_om) + j) : 0.f;
+        __syncthreads();
+    }
 
     const int li = (int)a.div_tpi.div((uint32_t)lane);     // item within the run
     const int chunk = lane - li * a.tpi;                    // channel chunk of the item
@@ -239,20 +377,32 @@ __global__ void __launch_bounds__(kDcnMaxThreads, 1) dcn_fwd_kernel(const DcnArg
         const int nitems = min(a.run_items, row_items - i0);
         const long long item_base = ((long long)n * a.Ho + oy) * row_items + i0;
 
-        const T* offp;
-        const T* maskp;
+        const OT* offp;
+        const OT* maskp;
         if (staged) {
             __syncwarp();                                    // previous run's reads are done
-            warp_stage(s_off, static_cast<const T*>(a.offset) + item_base * K * 2,
-                       nitems * K * 2, lane);
-            warp_stage(s_mask, static_cast<const T*>(a.mask) + item_base * K, nitems * K,
-                       lane);
+            if constexpr (FUSED) {
+                const int rows = (a.J + 15) & ~15;
+                const T* Ws = reinterpret_cast<const T*>(wsm);
+                const float* bs = reinterpret_cast<const float*>(
+                    wsm + ((rows * fused_w_stride(a.C) * (int)sizeof(T) + 15) & ~15));
+                const T* xrow = static_cast<const T*>(a.x) + ((long long)n * a.H + oy) * a.W * a.C;
+                fused_front_end<T>(xrow, i0 / a.G, (nitems + a.G - 1) / a.G, a.C, a.J, a.G * K,
+                                   Ws, bs, s_off, s_mask, lane);
+            } else {
+                warp_stage(s_off, static_cast<const T*>(a.offset) + item_base * K * 2,
+                           nitems * K * 2, lane);
+                warp_stage(s_mask, static_cast<const T*>(a.mask) + item_base * K, nitems * K,
+                           lane);
+            }
             __syncwarp();
             offp = s_off + li * K * 2;
             maskp = s_mask + li * K;
         } else {
-            offp = static_cast<const T*>(a.offset) + (item_base + li) * K * 2;
-            maskp = static_cast<const T*>(a.mask) + (item_base + li) * K;
+            offp = reinterpret_cast<const OT*>(static_cast<const T*>(a.offset) +
+                                               (item_base + li) * K * 2);
+            maskp = reinterpret_cast<const OT*>(static_cast<const T*>(a.mask) +
+                                                (item_base + li) * K);
         }
         if (li >= nitems) continue;
 
@@ -267,14 +417,14 @@ __global__ void __launch_bounds__(kDcnMaxThreads, 1) dcn_fwd_kernel(const DcnArg
         // DCNv3: stable softmax of the group's K logits
         float zmax = 0.f, inv_sum = 1.f;
         if constexpr (SOFTMAX) {
-            zmax = Elem<T>::one(maskp);
-            for (int k = 1; k < K; ++k) zmax = fmaxf(zmax, Elem<T>::one(maskp + k));
+            zmax = Elem<OT>::one(maskp);
+            for (int k = 1; k < K; ++k) zmax = fmaxf(zmax, Elem<OT>::one(maskp + k));
             float s = 0.f;
-            for (int k = 0; k < K; ++k) s += expf(Elem<T>::one(maskp + k) - zmax);
+            for (int k = 0; k < K; ++k) s += expf(Elem<OT>::one(maskp + k) - zmax);
             inv_sum = 1.f / s;
         }
         auto modulation = [&](int k) {
-            const float z = Elem<T>::one(maskp + k);
+            const float z = Elem<OT>::one(maskp + k);
             if constexpr (SOFTMAX) return expf(z - zmax) * inv_sum;
             return z;
         };
@@ -294,7 +444,7 @@ __global__ void __launch_bounds__(kDcnMaxThreads, 1) dcn_fwd_kernel(const DcnArg
         auto geometry = [&]() {
             const int k = nix * kh + niy;
             float dx, dy;
-            load_pair<T>(offp + 2 * k, dx, dy);
+            load_pair<OT>(offp + 2 * k, dx, dy);
             const TapGeom t = tap_geometry(a, bx + nix * a.dil, by + niy * a.dil, dx, dy,
                                            modulation(k));
             if (++niy == kh) {

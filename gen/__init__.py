@@ -117,6 +117,46 @@ class DynWorkload:
 
 
 @dataclass(frozen=True)
+class FusedWorkload:
+    """DCNv4 core fed by its merged offset / mask linear (stride 1)."""
+    name: str
+    N: int
+    H: int
+    W: int
+    C: int
+    G: int
+    kh: int = 3
+    kw: int = 3
+    pad: int = 1
+    dil: int = 1
+    dtype: str = "f16"
+    offset_sigma: float = 2.0
+
+    @property
+    def K(self):
+        return self.kh * self.kw
+
+    @property
+    def J(self):
+        return self.G * self.K * 3
+
+    @property
+    def D(self):
+        return self.C // self.G
+
+    def taps(self):
+        return self.N * self.H * self.W * self.G * self.K
+
+    def pixels(self):
+        return self.N * self.H * self.W
+
+    def compulsory_bytes(self):
+        """x and out once, the linear's weights and bias once."""
+        es = DTYPES[self.dtype].itemsize
+        return (2 * self.pixels() * self.C + self.J * (self.C + 1)) * es
+
+
+@dataclass(frozen=True)
 class MsdaWorkload:
     name: str
     N: int
@@ -182,6 +222,9 @@ WORKLOADS = {w.name: w for w in [
     # DCNv4 fp16 at dense-prediction resolution with heavy-tailed offsets
     DcnWorkload("dcnv4_f16_2x200x320x64_g4", N=2, H=200, W=320, C=64, G=4, dtype="f16",
                 offset_sigma=8.0),
+    # the headline shape through the fused front end (merged offset / mask
+    # linear on the tensor cores feeding the sampler)
+    FusedWorkload("dcnv4_fused_f16_64x56x56x64_g4", N=64, H=56, W=56, C=64, G=4),
     # ContMix core (dynamic K x K kernels, softmax) at the first-stage shape:
     # the 7 x 7 and 13 x 13 kernel sizes of the OverLoCK networks
     DynWorkload("contmix_f16_64x56x56x64_g4_k7", N=64, H=56, W=56, C=64, G=4, K=7),
@@ -263,6 +306,21 @@ def grad_out(shape, dtype, seed=0):
     forward inputs of the same seed are unchanged."""
     rng = np.random.default_rng([seed, 0x6772])
     return _round(rng.normal(0.0, 1.0, size=tuple(shape)), dtype)
+
+
+def front_end_inputs(w, seed=0):
+    """x ~U[-1,1]; w_om ~N(0, s^2) with s chosen so that the linear's offsets
+    have std offset_sigma px and its masks std 1 (x has variance 1/3 per
+    channel); b_om ~N(0, 0.25).  CPU tensors."""
+    rng = np.random.default_rng(seed)
+    x = rng.uniform(-1.0, 1.0, size=(w.N, w.H, w.W, w.C))
+    n_off = w.G * w.K * 2
+    s_off = np.sqrt(3.0 * w.offset_sigma ** 2 / w.C)
+    s_mask = np.sqrt(3.0 / w.C)
+    w_om = np.concatenate([rng.normal(0.0, s_off, size=(n_off, w.C)),
+                           rng.normal(0.0, s_mask, size=(w.J - n_off, w.C))], axis=0)
+    b_om = rng.normal(0.0, 0.5, size=(w.J,))
+    return {"x": _round(x, w.dtype), "w_om": _round(w_om, w.dtype), "b_om": _round(b_om, w.dtype)}
 
 
 def msda_ref_inputs(w, seed=0):

@@ -131,6 +131,32 @@ DCN_API int msda_forward(const void* value, const int64_t* spatial_shapes,
                  int L, int K, int dtype, void* stream);
 
 /*
+ * dcnv4_fused_forward - DCNv4 core fed by its merged offset / mask linear.
+ *
+ * Defined by the "DCNv4" note, "1. Remove Softmax" (one linear layer gives
+ * each location its G*K offset pairs and G*K modulation scalars, used without
+ * a softmax) and the passages of dcn_forward.  For every pixel p:
+ *   om[p][j] = sum_c w_om[j][c] * x[p][c] + b_om[j],  j < J = G * K * 3
+ *   offset[p][g][k][c2] = om[p][(g*K + k)*2 + c2],  mask[p][g][k] = om[p][2GK + g*K + k]
+ *   out = dcn_forward(x, offset, mask) with stride 1 and softmax_flag 0.
+ * The offsets and masks are computed per warp on the tensor cores (16-bit
+ * inputs, float32 accumulation), kept in float32 in shared memory and never
+ * written to global memory.
+ *
+ * Layouts: x [N][H][W][C], w_om [J][C], b_om [J] (or NULL for no bias),
+ * out [N][H][W][C]; all 16-bit (f16 or bf16).
+ * Limits: dtype f16 / bf16 (f32: DCN_ERR_UNSUPPORTED); odd kh, kw with
+ * pad * 2 == dil * (kh - 1) == dil * (kw - 1) (the output keeps the input
+ * size); C a multiple of 16, at most 128; a warp's run of (pixel, group) items must hold
+ * whole pixels (32 / TPI a multiple of G); the limits of dcn_forward.
+ * Errors: as dcn_forward; DCN_ERR_MISALIGNED unless x and out are 4-byte
+ * aligned and w_om, b_om aligned to the element size.
+ */
+DCN_API int dcnv4_fused_forward(const void* x, const void* w_om, const void* b_om, void* out,
+                 int N, int H, int W, int C, int G, int kh, int kw, int pad, int dil,
+                 int dtype, void* stream);
+
+/*
  * msda_forward_points - msda_forward fed from reference points or boxes.
  *
  * Defined by "Deformable DETR: Learn Where to Read", "A reference links
