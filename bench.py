@@ -49,8 +49,8 @@ FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_write.sum per launch, headline workload), with the hash of the
 # forward kernel's sources it was taken on; reported as null once they change.
 NCU_TRAFFIC = {
-    "source_sha256": "6153b12ff5da32abec3aa2b88a07b2211c9d6bd6b43e0667a7e965e94f9e7a64",
-    "bytes_per_launch": 69196544 + 3538944,   # DRAM read + write, one headline launch
+    "source_sha256": "6d556fb9616c39b7868e0c7d55395ae33b1bcfcba3da14795739eb6a254e8dc1",
+    "bytes_per_launch": 69190144 + 3826688,   # DRAM read + write, one headline launch
 }
 
 # What the forward DCN launch depends on: its device code, and in the C
