@@ -11,14 +11,14 @@
 //
 // Work decomposition (one CTA = one tile of TH rows x 32 columns, one group,
 // one 32-byte channel chunk):
-//   thread  = 4 consecutive output columns (P = 4) of one row, CPT channels
-//             (32 bytes: 16 fp16 / bf16 or 8 fp32); 8 threads span the tile's
-//             32 columns, so a warp covers 4 rows.
+//   thread  = P = 2 consecutive output columns of one row, CPT channels
+//             (32 bytes: 16 fp16 / bf16 or 8 fp32); 16 threads span the tile's
+//             32 columns, so a warp covers 2 rows.
 //   window  = rows [y0 - K/2, y0 + TH - 1 + K/2], columns likewise, copied with
 //             cp.async (zero-filled outside the map, all copies in flight at
 //             once); pixel c of a window row sits at byte c*32 + (c/4)*16, so
-//             the 32-byte loads of a warp (threads 4 columns apart) spread over
-//             all banks.
+//             the 32-byte loads of a warp (threads 2 columns apart) spread over
+//             the banks.
 //   weights = one kernel row (ky) at a time: the K numbers of every location
 //             are copied with 16-byte cp.async blocks (from the block that holds
 //             the first number, the last copy clipped to the row's end) into a
@@ -31,15 +31,15 @@
 //             running sum and the owner's accumulators are rescaled when the
 //             maximum grows; the output is divided by the sum at the end.
 // Per kernel row the thread slides along x: each window pixel it loads (two
-// 16-byte shared loads, widened once) is multiplied into the up to four
-// outputs whose taps cover it, with packed FFMA2 into float32 accumulators.
+// 16-byte shared loads, widened once) is multiplied into the up to P outputs
+// whose taps cover it, with packed FFMA2 into float32 accumulators.
 #pragma once
 
 #include "common.cuh"
 
 namespace dcnb {
 
-constexpr int kDynP = 4;            // output columns per thread
+constexpr int kDynP = 2;            // output columns per thread (2: measured faster than 4, more warps)
 constexpr int kDynTileW = 32;       // output columns per tile
 constexpr int kDynSegs = kDynTileW / kDynP;
 constexpr int kDynMaxK = 31;
@@ -127,9 +127,11 @@ __global__ void __launch_bounds__(256) dynconv_fwd_kernel(const DynArgs a) {
     const int w_col = a.G * KK;
     const int w_row = a.W * w_col;
     auto in_map = [&](int row, int col) { return y0 + row < a.H && x0 + col < a.W; };
-    // slot of location (row, col): ordered [col % 4][row][col / 4], so that the
+    // slot of location (row, col): ordered [col % P][row][col / P], so that the
     // owners of one column offset read consecutive slots
-    auto slot = [&](int row, int col) { return ((col & 3) * TH + row) * kDynSegs + (col >> 2); };
+    auto slot = [&](int row, int col) {
+        return ((col % kDynP) * TH + row) * kDynSegs + col / kDynP;
+    };
 
     // Copy kernel row ky of every location of the tile into raw buffer `buf`:
     // whole 16-byte blocks from the block holding the row's first number,
