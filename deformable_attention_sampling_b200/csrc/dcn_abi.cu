@@ -1087,6 +1087,8 @@ int msda_backward(const void* value, const int64_t* spatial_shapes, const int64_
     a.div_M = make_div((uint32_t)M);
     a.div_Lq = make_div((uint32_t)(Lq > 0 ? Lq : 1));
     a.div_tpi = make_div((uint32_t)tpi);
+    a.ref = nullptr;
+    a.vr = nullptr;
     b.grad_out = grad_out;
     b.grad_loc = grad_loc;
     b.grad_attn = grad_attn;

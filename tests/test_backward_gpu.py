@@ -253,3 +253,21 @@ def test_msda_backward_launches_and_repeat():
     check_msda(first, ref, "first")
     check_msda(second, ref, "second")
     assert torch.equal(first[1], second[1]) and torch.equal(first[2], second[2])
+
+
+def test_msda_backward_far_and_nan_locations():
+    """Locations far outside every level, and NaN ones, get zero location and
+    weight gradients and add nothing to grad_value; the rest match the oracle."""
+    w = gen.MsdaWorkload("far", N=1, M=2, D=16, shapes=((6, 8), (3, 4)), K=2, Lq=9,
+                         dtype="f32", offset_sigma=2.0)
+    inp = msda_problem(w, seed=14)
+    loc = inp["loc"].clone()
+    loc[0, 0, 0, 0, 0] = torch.tensor([40.0, -35.0])
+    loc[0, 1, 1, 1, 1, 0] = float("nan")
+    inp["loc"] = loc
+    gv, gl, ga = ref_msda_bwd(inp)
+    bad = ~np.isfinite(gl).all(axis=-1)
+    gl[bad] = 0.0
+    ga[bad] = 0.0
+    assert bad.sum() == 1 and np.isfinite(gv).all()
+    check_msda(run_msda_bwd(inp), (gv, gl, ga), "far / nan")

@@ -95,3 +95,13 @@ def test_dynconv_empty_batch():
     out = dcnb.dynconv(x, wt, 3)
     assert dcnb.dcn_launch_count() == before and out.shape == x.shape
     assert np.prod(out.shape) == 0
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16", "f32"])
+def test_dynconv_one_by_one_softmax_is_the_identity(dt):
+    """K = 1 with the softmax: every weight is exactly 1, so out == x bit for bit."""
+    C = 16 if dt != "f32" else 8
+    w = gen.DynWorkload("k1", N=2, H=5, W=37, C=C, G=1, K=1, dtype=dt)
+    inp = gen.dynconv_inputs(w, seed=13)
+    out = run(inp, w)
+    assert torch.equal(out.cpu(), inp["x"])

@@ -85,3 +85,15 @@ def test_reference_variant_validation():
                                  inp["reference"], 3, None, inp["offsets"], inp["attn"], out,
                                  1, 3, 2, 8, 1, 2, 0)
     assert e.value.status == dcnb.DCN_ERR_INVALID_ARG
+
+
+def test_mask_value_rows_not_multiple_of_16_bytes():
+    """M * D * 4 = 36 bytes per row: the element-wise path, out of place and in place."""
+    N, S, M, D = 2, 11, 3, 3
+    value = torch.randn(N, S, M, D, device=DEV)
+    mask = torch.rand(N, S, device=DEV) < 0.4
+    expect = value.masked_fill(mask[:, :, None, None], 0.0)
+    assert torch.equal(dcnb.mask_value(value, mask), expect)
+    dcnb.mask_value(value, mask, out=value)
+    torch.cuda.synchronize()
+    assert torch.equal(value, expect)
