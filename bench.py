@@ -49,7 +49,7 @@ FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_write.sum per launch, headline workload), with the hash of the
 # forward kernel's sources it was taken on; reported as null once they change.
 NCU_TRAFFIC = {
-    "source_sha256": "6d556fb9616c39b7868e0c7d55395ae33b1bcfcba3da14795739eb6a254e8dc1",
+    "source_sha256": "4759a5db507e1eb4cf2c92f0e46ac3da631aa04d770c1be48ca6718f61af10c5",
     "bytes_per_launch": 69190144 + 3826688,   # DRAM read + write, one headline launch
 }
 

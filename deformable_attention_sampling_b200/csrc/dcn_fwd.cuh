@@ -29,8 +29,10 @@
 // Channels accumulate in float32 with packed FFMA2; the result is rounded once
 // and stored with one streaming vector store.
 //
-// No tensor cores: the work is a gather and a weighted sum, not a contraction.
-// The binding limit is the SM's L1 data path for scattered 32-byte gathers.
+// The sampler uses no tensor cores: the work is a gather and a weighted sum,
+// not a contraction.  The binding limit is the SM's L1 data path for
+// scattered 32-byte gathers.  Only the FUSED variant's front end (the merged
+// offset / mask linear) is a contraction, and it runs on the tensor cores.
 #pragma once
 
 #include <type_traits>
