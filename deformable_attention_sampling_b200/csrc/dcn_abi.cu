@@ -276,6 +276,21 @@ const void* dcn_fused_kernel_vb(int vb, int kh, int kw) {
     }
 }
 
+template <typename T, int KT>
+const void* dynconv_kernel_k(int softmax) {
+    return softmax ? (const void*)dcnb::dynconv_fwd_kernel<T, true, KT>
+                   : (const void*)dcnb::dynconv_fwd_kernel<T, false, KT>;
+}
+
+template <typename T>
+const void* dynconv_kernel_for(int softmax, int K) {
+    switch (K) {
+        case 7: return dynconv_kernel_k<T, 7>(softmax);
+        case 13: return dynconv_kernel_k<T, 13>(softmax);
+        default: return dynconv_kernel_k<T, 0>(softmax);
+    }
+}
+
 // ---------------------------------------------------------------- MSDA -----
 
 template <typename T, int REF>
@@ -973,7 +988,9 @@ int dynconv_forward(const void* x, const void* weights, void* out, int N, int H,
     a.win_rows = th + K - 1;
     a.row_bytes = dcnb::dyn_row_bytes(dcnb::kDynTileW + K - 1);
     a.xs_bytes = a.win_rows * a.row_bytes;
-    a.ws_bytes = ((K * dcnb::dyn_wstride(th) * 4) + 15) & ~15;
+    // the compiled kernel sizes keep their weights in registers: no slots
+    const bool fixed_k = K == 7 || K == 13;
+    a.ws_bytes = fixed_k ? 0 : ((K * dcnb::dyn_wstride(th) * 4) + 15) & ~15;
     const int raw_bytes = 2 * th * dcnb::kDynTileW * dcnb::dyn_slot_bytes(K, es);   // two buffers
     const int smem = a.xs_bytes + a.ws_bytes + raw_bytes;
     if (smem > kMaxBwdSmemBytes) return DCN_ERR_UNSUPPORTED;
@@ -982,18 +999,9 @@ int dynconv_forward(const void* x, const void* weights, void* out, int N, int H,
 
     const void* fn = nullptr;
     switch (dtype) {
-        case DCN_F32:
-            fn = softmax_flag ? (const void*)dcnb::dynconv_fwd_kernel<float, true>
-                              : (const void*)dcnb::dynconv_fwd_kernel<float, false>;
-            break;
-        case DCN_F16:
-            fn = softmax_flag ? (const void*)dcnb::dynconv_fwd_kernel<__half, true>
-                              : (const void*)dcnb::dynconv_fwd_kernel<__half, false>;
-            break;
-        case DCN_BF16:
-            fn = softmax_flag ? (const void*)dcnb::dynconv_fwd_kernel<__nv_bfloat16, true>
-                              : (const void*)dcnb::dynconv_fwd_kernel<__nv_bfloat16, false>;
-            break;
+        case DCN_F32: fn = dynconv_kernel_for<float>(softmax_flag, K); break;
+        case DCN_F16: fn = dynconv_kernel_for<__half>(softmax_flag, K); break;
+        case DCN_BF16: fn = dynconv_kernel_for<__nv_bfloat16>(softmax_flag, K); break;
         default: break;
     }
     if (!fn) return DCN_ERR_UNSUPPORTED;

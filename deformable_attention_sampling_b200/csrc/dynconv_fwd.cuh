@@ -75,7 +75,11 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t 
 // holds ceil((K * es + 15) / 16) whole blocks.
 __host__ __device__ inline int dyn_slot_bytes(int K, int es) { return ((K * es + 15 + 15) / 16) * 16; }
 
-template <typename T, bool SOFTMAX>
+// KT > 0: the kernel size fixed at compile time (the workloads' 7 and 13).
+// Each thread then keeps its locations' weights of the current kernel row in
+// registers (no float32 weight slots in shared memory, so more CTAs fit on an
+// SM) and the sliding loop unrolls.  KT = 0: any odd K up to kDynMaxK.
+template <typename T, bool SOFTMAX, int KT = 0>
 __global__ void __launch_bounds__(256) dynconv_fwd_kernel(const DynArgs a) {
     constexpr int CPT = 32 / (int)sizeof(T);
     constexpr int es = (int)sizeof(T);
@@ -83,7 +87,7 @@ __global__ void __launch_bounds__(256) dynconv_fwd_kernel(const DynArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int TH = a.th;
     const int NP = TH * kDynTileW;                  // locations of the tile
-    const int K = a.K, KK = K * K, r = K >> 1;
+    const int K = KT ? KT : a.K, KK = K * K, r = K >> 1;
     const int SB = dyn_slot_bytes(K, es);
     unsigned char* xs = smem;
     float* ws = reinterpret_cast<float*>(smem + a.xs_bytes);
@@ -174,6 +178,12 @@ __global__ void __launch_bounds__(256) dynconv_fwd_kernel(const DynArgs a) {
     }
     const int wstride = dyn_wstride(TH);
     float* wk = ws + row * (kDynTileW + 1) + col0;
+    float wreg[kDynP][KT ? KT : 1];   // KT > 0: this row's weights of the thread's locations
+    (void)wreg;
+    auto put_w = [&](int p, int kx, float v) {
+        if constexpr (KT > 0) wreg[p][kx] = v;
+        else wk[kx * wstride + p] = v;
+    };
 
     copy_row(0, 0);
     for (int ky = 0; ky < K; ++ky) {
@@ -190,7 +200,8 @@ __global__ void __launch_bounds__(256) dynconv_fwd_kernel(const DynArgs a) {
 #pragma unroll
         for (int p = 0; p < kDynP; ++p) {
             if (!mine[p]) {
-                for (int kx = 0; kx < K; ++kx) wk[kx * wstride + p] = 0.f;
+#pragma unroll
+                for (int kx = 0; kx < K; ++kx) put_w(p, kx, 0.f);
                 continue;
             }
             const int sk = (skew[p] + ky * K * es) & 15;
@@ -203,21 +214,24 @@ __global__ void __launch_bounds__(256) dynconv_fwd_kernel(const DynArgs a) {
                 mrun[p] = m;
                 const float ml = m * kLog2e;
                 float srow = 0.f;
+#pragma unroll
                 for (int kx = 0; kx < K; ++kx) {
                     const float e = exp2f(fmaf(Elem<T>::one(zr + kx), kLog2e, -ml));
                     srow += e;
-                    wk[kx * wstride + p] = e;
+                    put_w(p, kx, e);
                 }
                 ssum[p] = fmaf(ssum[p], sc, srow);
 #pragma unroll
                 for (int i = 0; i < CPT; ++i) acc[p][i] *= sc;
             } else {
-                for (int kx = 0; kx < K; ++kx) wk[kx * wstride + p] = Elem<T>::one(zr + kx);
+#pragma unroll
+                for (int kx = 0; kx < K; ++kx) put_w(p, kx, Elem<T>::one(zr + kx));
             }
         }
 
         // slide along the window row (row + ky) over columns col0 .. col0 + K + P - 2
         const unsigned char* xrow = xs + (row + ky) * a.row_bytes;
+#pragma unroll
         for (int j = 0; j < K + kDynP - 1; ++j) {
             const unsigned char* px = xrow + dyn_pixel_byte(col0 + j);
             uint32_t wv[8];
@@ -230,7 +244,10 @@ __global__ void __launch_bounds__(256) dynconv_fwd_kernel(const DynArgs a) {
 #pragma unroll
             for (int p = 0; p < kDynP; ++p) {
                 const int kx = j - p;
-                if (kx >= 0 && kx < K) axpy<CPT>(acc[p], wk[kx * wstride + p], f);
+                if (kx >= 0 && kx < K) {
+                    if constexpr (KT > 0) axpy<CPT>(acc[p], wreg[p][kx], f);
+                    else axpy<CPT>(acc[p], wk[kx * wstride + p], f);
+                }
             }
         }
     }
