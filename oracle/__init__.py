@@ -42,6 +42,8 @@ def bind(lib):
     lib.oracle_msda_backward.restype = ctypes.c_int
     lib.oracle_dynconv_forward.argtypes = [dp, dp, dp] + [L] * 6 + [ctypes.c_int]
     lib.oracle_dynconv_forward.restype = ctypes.c_int
+    lib.oracle_msda_locations.argtypes = [dp, L, dp, dp, lp, dp] + [L] * 5
+    lib.oracle_msda_locations.restype = ctypes.c_int
     return lib
 
 
@@ -197,23 +199,30 @@ def msda_locations_ref(spatial_shapes, reference, offsets, valid_ratios=None):
 
     reference [N, Lq, 2] points or [N, Lq, 4] boxes (cx, cy, w, h) in
     valid-image coordinates; offsets [N, Lq, M, L, K, 2]; valid_ratios
-    [N, L, 2] as (W_valid / W, H_valid / H), or None for all 1.  Applies
-    scalar.sampling_location_ref element by element -> loc [N, Lq, M, L, K, 2].
+    [N, L, 2] as (W_valid / W, H_valid / H), or None for all 1; spatial_shapes
+    [L, 2] as (H, W).  Runs the C loop oracle_msda_locations (point:
+    s = p r + dp / (W, H); box: s = c r + (dp / K) (w, h) r / 2)
+    -> loc [N, Lq, M, L, K, 2].
     """
     ref = _as_f64(reference)
     off = _as_f64(offsets)
-    shapes = np.asarray(spatial_shapes, dtype=np.int64)
+    shapes = np.ascontiguousarray(np.asarray(spatial_shapes, dtype=np.int64))
     N, Lq, M, L, K, _ = off.shape
-    vr = np.ones((N, L, 2)) if valid_ratios is None else _as_f64(valid_ratios)
-    loc = np.empty_like(off)
-    for n in range(N):
-        for q in range(Lq):
-            for m in range(M):
-                for l in range(L):
-                    wh = (float(shapes[l][1]), float(shapes[l][0]))
-                    for k in range(K):
-                        loc[n, q, m, l, k] = scalar.sampling_location_ref(
-                            ref[n, q], off[n, q, m, l, k], wh, K, vr[n, l])
+    ref_dim = ref.shape[-1]
+    assert ref.shape == (N, Lq, ref_dim), "reference has the wrong shape"
+    assert shapes.shape == (L, 2), "spatial_shapes has the wrong shape"
+    loc = np.zeros_like(off)
+    if valid_ratios is None:
+        vr_ptr = None
+    else:
+        vr = _as_f64(valid_ratios)
+        assert vr.shape == (N, L, 2), "valid_ratios has the wrong shape"
+        vr_ptr = _ptr(vr)
+    rc = _load().oracle_msda_locations(_ptr(ref), ref_dim, vr_ptr, _ptr(off),
+                                       _ptr(shapes, ctypes.c_longlong), _ptr(loc), N, Lq, M,
+                                       L, K)
+    if rc != 0:
+        raise ValueError("oracle_msda_locations rejected its arguments")
     return loc
 
 

@@ -24,7 +24,10 @@
  *        between cells" and helper 2 (x = u W - 1/2, y = v H - 1/2, tent weights
  *        (1-|x-i|)+ (1-|y-j|)+ over the four floor/ceil neighbours, zero
  *        outside, no clamping, no renormalisation) and helper 3 (h_m = sum over
- *        levels and points of A_mlk times the sampled value).
+ *        levels and points of A_mlk times the sampled value); "A reference links
+ *        resolutions without equating their pixels" (point and box references
+ *        scaled by the level's valid ratio, offsets divided by the level size
+ *        or scaled by the box size).
  *   [P5] "OverLoCK" note, "ContMix: Put the Whole Image into the Kernel"
  *        (steps 4-5: a softmax turns each location's K^2 numbers into its own
  *        K x K kernel per channel group, which is applied to the zero-padded
@@ -212,6 +215,61 @@ int oracle_msda_forward(const double *value, const long long *shapes,
             }
         }
         out[(n * Lq + q) * M * D + h * D + c] = acc;
+    }
+    return 0;
+}
+
+/*
+ * Sampling locations of the reference-point variants, [P4] "A reference links
+ * resolutions without equating their pixels" (the point formula and the
+ * remark that a box reference has its centre and size scaled by the level's
+ * valid ratio first) and its step "Translate a reference into each sampling
+ * frame" (the box replaces the offset term by (dp / K) (w, h) r_l / 2).
+ * Everything is componentwise, x with widths and y with heights:
+ *   point p = (px, py):        s = p r_l + dp / (W_l, H_l)
+ *   box (cx, cy, w, h):        s = (cx, cy) r_l + (dp / K) (w, h) r_l / 2
+ * with r_l = (W_valid / W_l, H_valid / H_l) of the image and level (1 when
+ * valid_ratios is NULL).  Nothing is clamped.
+ *   reference     [N][Lq][ref_dim]      ref_dim 2 (point) or 4 (box)
+ *   valid_ratios  [N][L][2]             (x ratio, y ratio), or NULL
+ *   offsets       [N][Lq][M][L][K][2]   dp = (dx, dy)
+ *   shapes        [L][2]                (H_l, W_l)
+ *   loc           [N][Lq][M][L][K][2]   out: normalised (u, v)
+ * Returns 0, or -1 on a bad argument.
+ */
+int oracle_msda_locations(const double *reference, long ref_dim, const double *valid_ratios,
+                          const double *offsets, const long long *shapes, double *loc,
+                          long N, long Lq, long M, long L, long K)
+{
+    if (N < 0 || Lq < 0 || M <= 0 || L <= 0 || K <= 0 || (ref_dim != 2 && ref_dim != 4))
+        return -1;
+    for (long l = 0; l < L; ++l)
+        if (shapes[2 * l] <= 0 || shapes[2 * l + 1] <= 0)
+            return -1;
+    for (long n = 0; n < N; ++n)
+    for (long q = 0; q < Lq; ++q)
+    for (long h = 0; h < M; ++h)
+    for (long l = 0; l < L; ++l) {
+        const double *ref = reference + (n * Lq + q) * ref_dim;
+        double level_h = (double)shapes[2 * l];
+        double level_w = (double)shapes[2 * l + 1];
+        double ratio_x = valid_ratios ? valid_ratios[(n * L + l) * 2] : 1.0;
+        double ratio_y = valid_ratios ? valid_ratios[(n * L + l) * 2 + 1] : 1.0;
+        for (long k = 0; k < K; ++k) {
+            long t = (((n * Lq + q) * M + h) * L + l) * K + k;
+            double dx = offsets[2 * t];
+            double dy = offsets[2 * t + 1];
+            double u, v;
+            if (ref_dim == 2) {
+                u = ref[0] * ratio_x + dx / level_w;
+                v = ref[1] * ratio_y + dy / level_h;
+            } else {
+                u = ref[0] * ratio_x + (dx / (double)K) * ref[2] * ratio_x / 2.0;
+                v = ref[1] * ratio_y + (dy / (double)K) * ref[3] * ratio_y / 2.0;
+            }
+            loc[2 * t] = u;
+            loc[2 * t + 1] = v;
+        }
     }
     return 0;
 }

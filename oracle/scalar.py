@@ -8,9 +8,11 @@ Sources (page title, section):
   "InternImage: Deformable Convolutions at Scale" ch.2 (bilinear read),
       ch.3 (softmax over the K taps, worked example with K = 3).
   "DCNv4", "1. Remove Softmax" (modulation used as given).
-  "Deformable DETR: Learn Where to Read", helper 1 (reference to sampling
-      location), helper 2 (align_corners=False sample), helper 3 (joint
-      softmax over levels and points of one head, aggregation).
+  "Deformable DETR: Learn Where to Read", "A reference links resolutions
+      without equating their pixels" (point reference to sampling location),
+      "A learned location can fall between cells" (normalised to pixel-index
+      coordinates), helper 3 (joint softmax over levels and points of one
+      head, aggregation).
 """
 import math
 
@@ -48,18 +50,12 @@ def bilinear_pixel(grid, px, py):
 def bilinear_normalized(grid, u, v):
     """align_corners=False sample of grid at normalised (u, v), zero padding.
 
-    x = u W - 1/2, y = v H - 1/2; each of the four floor/ceil neighbours
-    weighs (1 - |x - col|)(1 - |y - row|) (Deformable DETR, helper 2).
+    Deformable DETR, "A learned location can fall between cells": the
+    normalised point maps to the pixel-index point (u W - 1/2, v H - 1/2),
+    which is then read with the pixel bilinear above (the page's tent weights
+    over the four floor/ceil neighbours are the same four corner weights).
     """
-    height, width = len(grid), len(grid[0])
-    x = u * width - 0.5
-    y = v * height - 0.5
-    total = 0.0
-    for row in (math.floor(y), math.floor(y) + 1):
-        for col in (math.floor(x), math.floor(x) + 1):
-            if 0 <= row < height and 0 <= col < width:
-                total += (1 - abs(x - col)) * (1 - abs(y - row)) * grid[row][col]
-    return total
+    return bilinear_pixel(grid, u * len(grid[0]) - 0.5, v * len(grid) - 0.5)
 
 
 def softmax(logits):
@@ -92,35 +88,13 @@ def aggregate(values, weights):
 
 
 def sampling_location(reference, offset, shape_wh):
-    """2-D point reference to a normalised sampling location.
-
-    s = reference + offset / (W_l, H_l), componentwise, no clamping
-    (Deformable DETR, helper 1, point branch with valid ratio 1).
-    `shape_wh` is (width, height).
-    """
-    return [reference[0] + offset[0] / shape_wh[0],
-            reference[1] + offset[1] / shape_wh[1]]
-
-
-def sampling_location_ref(reference, offset, shape_wh, points, valid_ratio=(1.0, 1.0)):
-    """Point or box reference to a normalised location in a padded level.
+    """2-D point reference to a normalised sampling location, valid ratio 1.
 
     Deformable DETR, "A reference links resolutions without equating their
-    pixels" and helper 1: the reference is in valid-image coordinates and is
-    scaled by the level's valid ratio r = (W_valid / W, H_valid / H); a 2-D
-    point adds offset / (W, H); a 4-D box (cx, cy, w, h) adds
-    (offset / points) * (w, h) * r / 2 instead.  No clamping.
-    `shape_wh` is the padded level size (width, height).
+    pixels": s = p + dp / (W_l, H_l), componentwise, not clamped.
+    `shape_wh` is (width, height).
     """
-    out = []
-    for axis in range(2):
-        centre = reference[axis] * valid_ratio[axis]
-        if len(reference) == 4:
-            shift = offset[axis] / points * reference[axis + 2] * valid_ratio[axis] / 2.0
-        else:
-            shift = offset[axis] / shape_wh[axis]
-        out.append(centre + shift)
-    return out
+    return [p + d / size for p, d, size in zip(reference, offset, shape_wh)]
 
 
 def out_size(n_in, k, stride, pad, dil):
