@@ -47,21 +47,22 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic of the timed kernel from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum per launch, headline workload), with the hash of the
-# forward kernel's sources it was taken on; reported as null once they change.
+# files the headline launch is built from; reported as null once they change.
 NCU_TRAFFIC = {
     "source_sha256": "4759a5db507e1eb4cf2c92f0e46ac3da631aa04d770c1be48ca6718f61af10c5",
     "bytes_per_launch": 69190144 + 3826688,   # DRAM read + write, one headline launch
 }
 
-# What the forward DCN launch depends on: its device code, and in the C
-# interface the tile choice, the kernel dispatch and dcn_forward itself.
+# What the headline dcn_forward launch is built from: its device code and the
+# host code that validates, chooses the launch shape and dispatches it.
 FORWARD_SOURCES = [
     "deformable_attention_sampling_b200/csrc/common.cuh",
     "deformable_attention_sampling_b200/csrc/dcn_fwd.cuh",
+    "deformable_attention_sampling_b200/csrc/dcn_band.cuh",
+    "deformable_attention_sampling_b200/csrc/abi_common.cuh",
+    "deformable_attention_sampling_b200/csrc/abi_common.cu",
+    "deformable_attention_sampling_b200/csrc/abi_dcn_fwd.cu",
 ]
-FORWARD_ABI = "deformable_attention_sampling_b200/csrc/dcn_abi.cu"
-FORWARD_ABI_SPANS = [("struct TileShape {", "// ---------------------------------------------------------------- MSDA"),
-                     ("int dcn_forward(", "int msda_forward(")]
 
 
 def log(*a):
@@ -71,13 +72,11 @@ def log(*a):
 def kernel_source_hash():
     h = hashlib.sha256()
     for p in FORWARD_SOURCES:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
-    with open(os.path.join(ROOT, FORWARD_ABI)) as f:
-        text = f.read()
-    for begin, end in FORWARD_ABI_SPANS:
-        i = text.index(begin)
-        h.update(text[i:text.index(end, i)].encode())
+        path = os.path.join(ROOT, p)
+        if os.path.exists(path):
+            h.update(p.encode())
+            with open(path, "rb") as f:
+                h.update(f.read())
     return h.hexdigest()
 
 
@@ -574,22 +573,64 @@ def sample_of(w, n_images):
     return gen.scaled(w, N=1, Lq=max(1, min(w.queries, n_images * 64)))
 
 
-def cpu_baseline(w, budget_s=10.0, backward=False):
-    """The oracle as it stands, single-threaded, on a bounded sample of the
-    workload, repeated until about `budget_s` seconds of CPU work."""
+def _oracle_worker(task):
+    """One host process of the all-core leg: runs the oracle on its tasks
+    (each a bounded sample with its own seed) and returns its busy time and
+    taps.  Top-level so that a spawned process can import it."""
+    w, seeds, backward = task
+    busy, taps = 0.0, 0
+    for seed in seeds:
+        dt, t = oracle_step(w, seed=seed, backward=backward)
+        busy += dt
+        taps += t
+    return busy, taps
+
+
+def cpu_baseline(w, budget_s=10.0, backward=False, pool=None, cores=1):
+    """The oracle as it stands on a bounded sample of the workload.
+
+    Single-threaded: repeated until about budget_s / 2 seconds of CPU work.
+    All cores: `pool` (spawned processes, one per host core) runs the same
+    oracle on the same sample size, each process over its own seeds, about
+    budget_s / 2 seconds per process; the rate is all taps over the busiest
+    process's oracle time (input generation is outside the timed calls)."""
     s = sample_of(w, 8)
     total_t, total_taps, reps = 0.0, 0, 0
-    while total_t < budget_s or reps == 0:
+    while total_t < budget_s / 2 or reps == 0:
         dt, taps = oracle_step(s, seed=reps, backward=backward)
         total_t += dt
         total_taps += taps
         reps += 1
-    desc = (f"{reps} x oracle on {s.name} with N={s.N}" +
+    single = total_taps / total_t
+    what = (f"oracle on {s.name} with N={s.N}" +
             (f", Lq={s.queries}" if isinstance(s, gen.MsdaWorkload) else "") +
-            f" ({s.taps()} taps each), single thread, float64" +
-            (", backward" if backward else ""))
-    return {"value": total_taps / total_t, "unit": "taps/s", "cores": 1, "kind": "oracle",
-            "sample": desc, "host_cpus": os.cpu_count()}
+            f" ({s.taps()} taps each), float64" + (", backward" if backward else ""))
+    result = {"value": single, "unit": "taps/s", "cores": 1, "kind": "oracle",
+              "sample": f"{reps} x {what}, single thread", "host_cpus": os.cpu_count(),
+              "single_thread_value": single}
+    if pool is not None and cores > 1:
+        per = max(1, int(round(budget_s / 2 / (total_t / reps))))
+        tasks = [(s, [10_000 + c * per + i for i in range(per)], backward)
+                 for c in range(cores)]
+        parts = pool.map(_oracle_worker, tasks)
+        busiest = max(b for b, _ in parts)
+        taps_all = sum(t for _, t in parts)
+        result.update({
+            "value": taps_all / busiest, "cores": cores,
+            "sample": (f"{cores} processes x {per} x {what}, one process per host core "
+                       f"(rate = all taps / busiest process's oracle time); single thread: "
+                       f"{reps} x the same sample"),
+            "all_core_value": taps_all / busiest})
+    return result
+
+
+def start_oracle_pool(cores):
+    """Host processes for the all-core oracle leg, started with `spawn` (a
+    process forked after CUDA is initialised can hang)."""
+    import multiprocessing as mp
+    if cores <= 1:
+        return None
+    return mp.get_context("spawn").Pool(cores)
 
 
 # ------------------------------------------------------------------ main arms
@@ -621,6 +662,10 @@ def barrier(world, device):
 
 
 def run_b200(args):
+    # the all-core oracle leg's processes start before CUDA is initialised
+    pool = None
+    if int(os.environ.get("WORLD_SIZE", "1")) == 1:
+        pool = start_oracle_pool(os.cpu_count() or 1)
     world, rank, local = setup_distributed()
     device = torch.device(f"cuda:{local}")
     torch.cuda.set_device(device)
@@ -759,7 +804,11 @@ def run_b200(args):
             "clocks": sampler.summary(),
         }
         if world == 1:
-            result["cpu_baseline"] = cpu_baseline(w, backward=backward)
+            result["cpu_baseline"] = cpu_baseline(w, backward=backward, pool=pool,
+                                                  cores=os.cpu_count() or 1)
+    if pool is not None:
+        pool.close()
+        pool.join()
         if backward:
             result["pass"] = "backward"
             result["roofline"]["note"] = (
@@ -839,6 +888,33 @@ def metric_name(w, backward):
     return METRIC if w.name == gen.HEADLINE else f"sampled taps/s ({w.name})"
 
 
+def torchrun_command(args, port):
+    """The command that runs this benchmark as args.gpus ranks, one process
+    per GPU (torch.distributed.run on this node, rendezvous on 127.0.0.1)."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+           f"--master-port={port}", os.path.abspath(__file__), "--gpus", str(args.gpus),
+           "--steps", str(args.steps), "--warmup", str(args.warmup), "--impl", args.impl,
+           "--workload", args.workload, "--pass", args.pass_]
+    return cmd
+
+
+def launch_ranks(args):
+    """`--gpus N` without a launcher: start N ranks with torch.distributed.run
+    and return its exit status.  Fails loudly when the node has fewer GPUs."""
+    import socket
+    import subprocess
+    have = torch.cuda.device_count()
+    if have < args.gpus:
+        log(f"bench.py --gpus {args.gpus}: this node has {have} CUDA device(s); "
+            f"{args.gpus} are needed (one rank per GPU)")
+        return 2
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+    return subprocess.run(torchrun_command(args, port)).returncode
+
+
 def main():
     p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     p.add_argument("--gpus", type=int, default=1)
@@ -851,6 +927,13 @@ def main():
     args = p.parse_args()
     if args.warmup < 3:
         p.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        p.error("--gpus must be at least 1")
+    world = os.environ.get("WORLD_SIZE")
+    if world is None and args.gpus > 1:
+        sys.exit(launch_ranks(args))
+    if world is not None and int(world) != args.gpus:
+        p.error(f"--gpus {args.gpus} does not match the launcher's WORLD_SIZE={world}")
     result = run_reference(args) if args.impl == "reference" else run_b200(args)
     if result is not None:
         print(json.dumps(result), flush=True)

@@ -434,7 +434,7 @@ struct RoundArgs {
 };
 
 // p[0, n) = 0, with 16-byte stores on the aligned body.
-__global__ void __launch_bounds__(kUtilThreads) zero_f32_kernel(const ZeroArgs z) {
+static __global__ void __launch_bounds__(kUtilThreads) zero_f32_kernel(const ZeroArgs z) {
     float* p = z.p;
     const long long n = z.n;
     const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;

@@ -331,7 +331,7 @@ struct MaskArgs {
     int vec16;                   // 1: rows, value and out are 16-byte aligned
 };
 
-__global__ void __launch_bounds__(256) msda_mask_value_kernel(const MaskArgs m) {
+static __global__ void __launch_bounds__(256) msda_mask_value_kernel(const MaskArgs m) {
     const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long nthreads = (long long)gridDim.x * blockDim.x;
     const char* src = static_cast<const char*>(m.value);
