@@ -44,6 +44,8 @@ METRIC = ("sampled taps/s & achieved HBM GB/s vs peak "
 # footprint; the rate falls to about 30 B/clk when the footprint spills to L2).
 L1_GATHER_BYTES_PER_CLK = 58.0
 FALLBACK_HBM_GBS = 6650.0
+# Shared memory delivers 32 banks x 4 bytes per SM clock to conflict-free reads.
+SMEM_BYTES_PER_CLK = 128.0
 
 # DRAM traffic of the timed kernel from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum per launch, headline workload), with the hash of the
@@ -173,22 +175,27 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
 
 
-def on_chip_roofline(w, ms_per_launch, sampler, device):
+def on_chip_roofline(w, ms_per_launch, sampler, device, band=False):
     """The SM-side bound: every tap reads four corner vectors of D channels
-    through L1 (the kernels load all four, out-of-map ones from a clamped
-    address with zero weight).  Peak = the measured L1 gather rate x SMs x the
-    median SM clock sampled during the timed region."""
+    (the kernels load all four, out-of-map ones from a clamped address with
+    zero weight).  The gather kernel reads them through L1: peak = the
+    measured L1 rate of random 32-byte gathers x SMs x the median SM clock
+    sampled during the timed region.  The band kernel reads them from shared
+    memory with conflict-free 16-byte lanes: peak = 128 bytes per SM clock
+    (32 banks x 4 bytes) x SMs x the same clock."""
     es = gen.DTYPES[w.dtype].itemsize
     gathered = w.taps() * 4 * w.D * es
     achieved = gathered / (ms_per_launch * 1e-3) / 1e9
     clocks = sampler.summary()
     mhz = clocks["sm_mhz"] or clocks["sm_max_mhz"] or 1965
     sms = torch.cuda.get_device_properties(device).multi_processor_count
-    peak = L1_GATHER_BYTES_PER_CLK * sms * mhz * 1e6 / 1e9
-    return {"bound": "l1_gather", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "gathered_bytes_per_launch": gathered,
-            "peak_basis": f"{L1_GATHER_BYTES_PER_CLK:g} B/clk/SM measured random 32 B gathers"
-                          f" x {sms} SMs x {mhz} MHz"}
+    rate = SMEM_BYTES_PER_CLK if band else L1_GATHER_BYTES_PER_CLK
+    peak = rate * sms * mhz * 1e6 / 1e9
+    basis = ("128 B/clk/SM shared-memory bandwidth (32 banks x 4 B)" if band else
+             f"{L1_GATHER_BYTES_PER_CLK:g} B/clk/SM measured random 32 B gathers")
+    return {"bound": "smem" if band else "l1_gather", "achieved": achieved, "peak": peak,
+            "unit": "GB/s", "frac": achieved / peak, "gathered_bytes_per_launch": gathered,
+            "peak_basis": f"{basis} x {sms} SMs x {mhz} MHz"}
 
 
 def fma_roofline(w, ms_per_launch, sampler, device):
@@ -209,6 +216,8 @@ def fma_roofline(w, ms_per_launch, sampler, device):
 # ------------------------------------------------------------------ runners
 
 class DcnRunner:
+    algo = 0     # DCN_ALGO_AUTO; set from --algo
+
     def __init__(self, w, seed, device):
         import deformable_attention_sampling_b200 as dcnb
         self.dcnb = dcnb
@@ -229,12 +238,12 @@ class DcnRunner:
         w, lib = self.w, self.lib
         args = (s["x"].data_ptr(), s["offset"].data_ptr(), s["mask"].data_ptr(),
                 s["out"].data_ptr(), w.N, w.H, w.W, w.C, w.G, w.kh, w.kw, w.stride, w.pad,
-                w.dil, w.softmax_flag, self.code, stream)
+                w.dil, w.softmax_flag, self.code, self.algo, stream)
 
         def go():
-            st = lib.dcn_forward(*args)
+            st = lib.dcn_forward_algo(*args)
             if st != 0:
-                raise self.dcnb.DcnError(st, "dcn_forward")
+                raise self.dcnb.DcnError(st, "dcn_forward_algo")
         return go
 
     def inputs_of(self, s):
@@ -678,6 +687,20 @@ def run_b200(args):
 
     backward = args.pass_ == "backward"
     runner = make_runner(w, seed=1000 + rank, device=device, backward=backward)
+    band = False
+    if isinstance(runner, DcnRunner) and not backward:
+        runner.algo = dcnb.ALGO_CODES[args.algo]
+        # which kernel the timed calls run: the band kernel where it applies
+        if args.algo != "gather":
+            probe = runner.alloc_set()
+            band = dcnb.library().dcn_forward_algo(
+                probe["x"].data_ptr(), probe["offset"].data_ptr(), probe["mask"].data_ptr(),
+                probe["out"].data_ptr(), w.N, w.H, w.W, w.C, w.G, w.kh, w.kw, w.stride, w.pad,
+                w.dil, w.softmax_flag, runner.code, dcnb.DCN_ALGO_BAND,
+                int(torch.cuda.current_stream(device).cuda_stream)) == 0
+            torch.cuda.synchronize(device)
+            del probe
+        runner.kernel = "dcn_band_kernel" if band else "dcn_fwd_kernel"
     bytes_per_step = runner.bytes_per_step()
     l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
     n_sets = max(2, int(np.ceil(3 * l2_bytes / bytes_per_step)))
@@ -796,7 +819,8 @@ def run_b200(args):
                          if peak_src == "measured" else "fallback 6.65 TB/s"},
             "on_chip": (fma_roofline(w, ms_local / args.steps, sampler, device)
                         if isinstance(w, gen.DynWorkload)
-                        else on_chip_roofline(w, ms_local / args.steps, sampler, device)),
+                        else on_chip_roofline(w, ms_local / args.steps, sampler, device,
+                                              band=band)),
             "e2e": {"value": taps_total / (e2e_ms * 1e-3), "unit": "taps/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "steps": e2e_steps},
@@ -895,7 +919,7 @@ def torchrun_command(args, port):
            f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
            f"--master-port={port}", os.path.abspath(__file__), "--gpus", str(args.gpus),
            "--steps", str(args.steps), "--warmup", str(args.warmup), "--impl", args.impl,
-           "--workload", args.workload, "--pass", args.pass_]
+           "--workload", args.workload, "--pass", args.pass_, "--algo", args.algo]
     return cmd
 
 
@@ -924,6 +948,8 @@ def main():
     p.add_argument("--workload", default=gen.HEADLINE, choices=sorted(gen.WORKLOADS))
     p.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
                    help="time the forward call (default) or the backward call")
+    p.add_argument("--algo", default="auto", choices=["auto", "gather", "band"],
+                   help="DCN forward kernel (dcn_forward_algo); auto = dcn_forward")
     args = p.parse_args()
     if args.warmup < 3:
         p.error("--warmup must be at least 3")

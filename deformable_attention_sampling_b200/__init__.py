@@ -13,6 +13,10 @@ binding: it marshals pointers, sizes and streams and runs nothing itself.
     out = dcnb.dynconv(x, weights, K)        # ContMix core: per-pixel K x K kernels
 """
 from ._binding import (  # noqa: F401
+    ALGO_CODES,
+    DCN_ALGO_AUTO,
+    DCN_ALGO_BAND,
+    DCN_ALGO_GATHER,
     DCN_ERR_CUDA,
     DCN_ERR_INVALID_ARG,
     DCN_ERR_MISALIGNED,
@@ -28,12 +32,15 @@ from ._binding import (  # noqa: F401
     dcn_backward_static_scratch,
     dcn_backward_workspace_size,
     dcn_forward,
+    dcn_forward_algo,
+    dcn_forward_timeouts,
     dcn_grad,
     dcn_last_cuda_error,
     dcn_launch_count,
     dcn_output_size,
     dcnv4_fused,
     dcnv4_fused_forward,
+    dcnv4_fused_forward_algo,
     dcn_status_string,
     dcn_version,
     dtype_code,

@@ -21,6 +21,10 @@ DCN_ERR_UNSUPPORTED = -2
 DCN_ERR_MISALIGNED = -3
 DCN_ERR_CUDA = -4
 DTYPE_CODES = {"f32": 0, "f16": 1, "bf16": 2}
+DCN_ALGO_AUTO = 0
+DCN_ALGO_GATHER = 1
+DCN_ALGO_BAND = 2
+ALGO_CODES = {"auto": DCN_ALGO_AUTO, "gather": DCN_ALGO_GATHER, "band": DCN_ALGO_BAND}
 
 # every symbol include/dcn.h declares, with its ctypes signature
 _VP = ctypes.c_void_p
@@ -28,6 +32,8 @@ _I = ctypes.c_int
 _LL = ctypes.c_longlong
 SIGNATURES = {
     "dcn_forward": (_I, [_VP, _VP, _VP, _VP] + [_I] * 12 + [_VP]),
+    "dcn_forward_algo": (_I, [_VP, _VP, _VP, _VP] + [_I] * 13 + [_VP]),
+    "dcn_forward_timeouts": (_I, []),
     "msda_forward": (_I, [_VP] * 6 + [_I] * 7 + [_VP]),
     "msda_forward_points": (_I, [_VP] * 4 + [_I] + [_VP] * 4 + [_I] * 7 + [_VP]),
     "msda_mask_value": (_I, [_VP] * 3 + [_I] * 5 + [_VP]),
@@ -38,6 +44,7 @@ SIGNATURES = {
     "msda_backward": (_I, [_VP] * 10 + [_LL] + [_I] * 8 + [_VP]),
     "dynconv_forward": (_I, [_VP] * 3 + [_I] * 8 + [_VP]),
     "dcnv4_fused_forward": (_I, [_VP] * 4 + [_I] * 10 + [_VP]),
+    "dcnv4_fused_forward_algo": (_I, [_VP] * 4 + [_I] * 11 + [_VP]),
     "dcn_output_size": (_I, [_I] * 5),
     "dcn_status_string": (ctypes.c_char_p, [_I]),
     "dcn_last_cuda_error": (_I, []),
@@ -109,6 +116,25 @@ def dcn_forward(x, offset, mask, out, N, H, W, C, G, kh, kw, stride, pad, dil,
     _check(_load().dcn_forward(_ptr(x), _ptr(offset), _ptr(mask), _ptr(out), N, H, W, C, G,
                                kh, kw, stride, pad, dil, softmax_flag, dtype, _stream(stream)),
            "dcn_forward")
+
+
+def dcn_forward_algo(x, offset, mask, out, N, H, W, C, G, kh, kw, stride, pad, dil,
+                     softmax_flag, dtype, algo, stream=None):
+    """C dcn_forward_algo (algo: DCN_ALGO_AUTO / _GATHER / _BAND); raises
+    DcnError on a non-OK status."""
+    _check(_load().dcn_forward_algo(_ptr(x), _ptr(offset), _ptr(mask), _ptr(out), N, H, W, C,
+                                    G, kh, kw, stride, pad, dil, softmax_flag, dtype, algo,
+                                    _stream(stream)),
+           "dcn_forward_algo")
+
+
+def dcn_forward_timeouts():
+    """C dcn_forward_timeouts: the band kernel's timed-out-wait word on the
+    current device (0 when no wait ever ran out); synchronous."""
+    r = _load().dcn_forward_timeouts()
+    if r < 0:
+        raise DcnError(r, "dcn_forward_timeouts")
+    return r
 
 
 def msda_forward(value, spatial_shapes, level_start, sampling_loc, attn_w, out, N, Lq, M, D,
@@ -198,6 +224,15 @@ def dcnv4_fused_forward(x, w_om, b_om, out, N, H, W, C, G, kh, kw, pad, dil, dty
            "dcnv4_fused_forward")
 
 
+def dcnv4_fused_forward_algo(x, w_om, b_om, out, N, H, W, C, G, kh, kw, pad, dil, dtype, algo,
+                             stream=None):
+    """C dcnv4_fused_forward_algo; raises DcnError on a non-OK status."""
+    _check(_load().dcnv4_fused_forward_algo(_ptr(x), _ptr(w_om), _ptr(b_om), _ptr(out), N, H, W,
+                                            C, G, kh, kw, pad, dil, dtype, algo,
+                                            _stream(stream)),
+           "dcnv4_fused_forward_algo")
+
+
 def dcn_output_size(n_in, k, stride, pad, dil):
     return int(_load().dcn_output_size(n_in, k, stride, pad, dil))
 
@@ -235,11 +270,12 @@ def _require(cond, msg):
 
 
 def dcn(x, offset, mask, kh=3, kw=3, stride=1, pad=1, dil=1, softmax_flag=0, out=None,
-        stream=None):
-    """dcn_forward on torch CUDA tensors; allocates `out` when not given.
+        stream=None, algo="auto"):
+    """dcn_forward_algo on torch CUDA tensors; allocates `out` when not given.
 
     x [N, H, W, C], offset [N, Ho, Wo, G, K, 2], mask [N, Ho, Wo, G, K], all of
     one dtype (float32 / float16 / bfloat16), contiguous, on one CUDA device.
+    algo: "auto" (dcn_forward), "gather" or "band".
     """
     import torch
     _require(x.dim() == 4 and mask.dim() == 5 and offset.dim() == 6,
@@ -259,8 +295,9 @@ def dcn(x, offset, mask, kh=3, kw=3, stride=1, pad=1, dil=1, softmax_flag=0, out
         out = torch.empty((N, Ho, Wo, C), dtype=x.dtype, device=x.device)
     _require(tuple(out.shape) == (N, Ho, Wo, C) and out.dtype == x.dtype and out.is_contiguous(),
              "out has the wrong shape, dtype or layout")
-    dcn_forward(x, offset, mask, out, N, H, W, C, G, kh, kw, stride, pad, dil, softmax_flag,
-                dtype_code(x), stream)
+    _require(algo in ALGO_CODES, f"algo must be one of {sorted(ALGO_CODES)}")
+    dcn_forward_algo(x, offset, mask, out, N, H, W, C, G, kh, kw, stride, pad, dil,
+                     softmax_flag, dtype_code(x), ALGO_CODES[algo], stream)
     return out
 
 
@@ -422,9 +459,10 @@ def mask_value(value, mask, out=None, stream=None):
     return out
 
 
-def dcnv4_fused(x, w_om, b_om=None, groups=4, kh=3, kw=3, pad=1, dil=1, out=None, stream=None):
-    """dcnv4_fused_forward on torch CUDA tensors: x [N, H, W, C], w_om
-    [G*kh*kw*3, C], b_om [G*kh*kw*3] or None."""
+def dcnv4_fused(x, w_om, b_om=None, groups=4, kh=3, kw=3, pad=1, dil=1, out=None, stream=None,
+                algo="auto"):
+    """dcnv4_fused_forward_algo on torch CUDA tensors: x [N, H, W, C], w_om
+    [G*kh*kw*3, C], b_om [G*kh*kw*3] or None; algo "auto", "gather" or "band"."""
     import torch
     N, H, W, C = x.shape
     J = groups * kh * kw * 3
@@ -435,6 +473,7 @@ def dcnv4_fused(x, w_om, b_om=None, groups=4, kh=3, kw=3, pad=1, dil=1, out=None
                  "tensors must be contiguous CUDA tensors of one dtype")
     if out is None:
         out = torch.empty_like(x)
-    dcnv4_fused_forward(x, w_om, b_om, out, N, H, W, C, groups, kh, kw, pad, dil, dtype_code(x),
-                        stream)
+    _require(algo in ALGO_CODES, f"algo must be one of {sorted(ALGO_CODES)}")
+    dcnv4_fused_forward_algo(x, w_om, b_om, out, N, H, W, C, groups, kh, kw, pad, dil,
+                             dtype_code(x), ALGO_CODES[algo], stream)
     return out

@@ -78,6 +78,11 @@ def build(force=False, verbose=False, jobs=None):
         raise subprocess.CalledProcessError(1, "nvcc")
     cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *[_object(s) for s in SOURCES]]
     subprocess.run(cmd, check=True)
+    # the objects are not kept: every build compiles all units, and the
+    # library alone travels with the source tree
+    for s in SOURCES:
+        os.remove(_object(s))
+    os.rmdir(OBJ_DIR)
     return LIB
 
 

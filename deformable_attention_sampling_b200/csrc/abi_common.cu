@@ -21,6 +21,13 @@ int sm_count() {
 
 namespace {
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
 struct GridCacheEntry {
     const void* fn;
     int device;
@@ -106,6 +113,54 @@ int wave_size(const void* fn, int threads, int smem) {
 // L1 reuse dominates and tiles grow up to kDcnMaxWarps rows (one CTA per SM).
 constexpr int kSmallMapRows = 64;
 
+// Timeout word of the band kernel's bounded waits, one per device; its
+// device address is looked up once per device.
+__device__ unsigned int g_band_timeouts;
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_timeout_mutex;
+unsigned int* g_timeout_ptr[kMaxScratchDevices] = {};
+
+unsigned int* band_timeout_word() {
+    int device = 0;
+    if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxScratchDevices) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_timeout_mutex);
+    if (g_timeout_ptr[device] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_band_timeouts) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return nullptr;
+        }
+        g_timeout_ptr[device] = static_cast<unsigned int*>(p);
+    }
+    return g_timeout_ptr[device];
+}
+
+bool encode_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner,
+                    uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        (void)cudaGetLastError();
+    });
+    if (!g_encode) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t elem_strides[2] = {1, 1};
+    return g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                    2, const_cast<void*>(base), dims, strides, box, elem_strides,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 TileShape choose_tile(int N, int Ho, int runs, int kernel_extent, int sms, int cap,
                       int warps_by_regs) {
     const int kWarpsPerSmByRegs = warps_by_regs;   // forward: 80 registers per thread
@@ -158,6 +213,15 @@ const char* dcn_status_string(int status) {
         case DCN_ERR_CUDA: return "CUDA launch failed";
         default: return "unknown status";
     }
+}
+
+int dcn_forward_timeouts(void) {
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_band_timeouts, sizeof(v)) != cudaSuccess) {
+        g_last_cuda_error = (int)cudaGetLastError();
+        return DCN_ERR_CUDA;
+    }
+    return (int)(v & 0x7fffffffu);
 }
 
 int dcn_last_cuda_error(void) { return g_last_cuda_error; }

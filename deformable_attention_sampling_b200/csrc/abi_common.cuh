@@ -3,6 +3,7 @@
 // or synchronises; every launch goes to the caller's stream.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -125,5 +126,18 @@ struct TileShape {
 // SM holds at the kernel's register count.
 TileShape choose_tile(int N, int Ho, int runs, int kernel_extent, int sms, int cap,
                       int warps_by_regs);
+
+// A 2-D tensor map over a row-major matrix of 16-bit elements (`inner`
+// elements per row, `outer` rows, rows `row_bytes` apart) for tile loads of
+// box_inner x box_outer elements with the 128-byte swizzle; out-of-range box
+// elements read as zero.  The encoder comes from the driver through the
+// runtime's entry-point query (no link-time dependency on libcuda).  False on
+// any error.
+// Device address of the timeout word of the band kernels' bounded waits on
+// the current device (looked up once per device), or null.
+unsigned int* band_timeout_word();
+
+bool encode_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner,
+                    uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 
 }  // namespace dcnb_abi

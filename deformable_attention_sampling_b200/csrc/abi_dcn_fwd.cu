@@ -1,11 +1,105 @@
-// C interface of libdcn_b200.so: dcn_forward (argument checks, launch
-// shape, dispatch to the sm_100a DCN forward kernels).
+// C interface of libdcn_b200.so: dcn_forward and dcn_forward_algo (argument
+// checks, choice between the two forward kernels, launch shape, dispatch).
+//
+// Two kernels compute the same operator:
+//   - the band kernel (dcn_band.cuh): input rows staged in shared memory by
+//     bulk copies, conflict-free corner reads; 16-bit data, 16 channels per
+//     group, pixels of a multiple of 128 bytes, 16-byte aligned tensors and
+//     rows, and a band of rows that fits in shared memory;
+//   - the gather kernel (dcn_fwd.cuh): corners read through L1; every shape.
+// DCN_ALGO_AUTO takes the band kernel where it applies.
 #include "abi_common.cuh"
+#include "dcn_band.cuh"
 #include "dcn_fwd.cuh"
 
 using namespace dcnb_abi;
 
 namespace {
+
+constexpr int kBandMarginRows = 6;     // offset margin of the band, at most
+constexpr int kBandMinMarginRows = 2;
+constexpr int kBandSmemLimit = 227 * 1024;
+constexpr int kBandTargetItems = 14 * 32;   // items per step
+
+template <typename T>
+const void* band_kernel_for(int softmax, int kh, int kw) {
+    using namespace dcnb;
+    if (kh == 3 && kw == 3)
+        return softmax ? (const void*)dcn_band_kernel<T, true, 3>
+                       : (const void*)dcn_band_kernel<T, false, 3>;
+    return softmax ? (const void*)dcn_band_kernel<T, true, 0>
+                   : (const void*)dcn_band_kernel<T, false, 0>;
+}
+
+// Launch configuration of the band kernel for this call, or false when the
+// shape or the pointers do not qualify.
+bool band_config(const void* x, const void* offset, const void* mask, void* out, int N, int H,
+                 int W, int C, int G, int kh, int kw, int stride, int pad, int dil, int Ho,
+                 int Wo, int es, dcnb::BandArgs* a, int* smem, int* threads) {
+    const int D = C / G;
+    const int K = kh * kw;
+    if (es != 2 || D != 16 || (C * es) % 128 != 0) return false;
+    if ((((uintptr_t)x | (uintptr_t)offset | (uintptr_t)mask | (uintptr_t)out) % 16) != 0)
+        return false;
+    const long long row_bytes = (long long)W * C * es;
+    const long long off_row = (long long)Wo * G * K * 2 * es;
+    const long long mask_row = (long long)Wo * G * K * es;
+    if (off_row % 16 != 0 || mask_row % 16 != 0) return false;
+    const long long row_items = (long long)Wo * G;
+    const int runs_per_row = (int)((row_items + 31) / 32);
+    int th = (int)((kBandTargetItems + row_items - 1) / row_items);
+    th = std::max(1, std::min(th, std::min(4, Ho)));
+    const int warps = std::min(dcnb::kBandMaxConsumerWarps, th * runs_per_row);
+    const long long stage = (th * (off_row + mask_row) + 127) / 128 * 128;
+    for (int margin = kBandMarginRows; margin >= kBandMinMarginRows; --margin) {
+        if (pad > margin + (kh - 1) * dil) break;   // every band must meet the map
+        const int band = dcnb::band_rows(th, stride, kh, dil, margin);
+        const int band_in_map = std::min(band, H);
+        long long ring = band + (long long)(dcnb::kBandStages - 1) * th * stride;
+        ring = std::min(ring, 2LL * H);
+        ring = std::max<long long>(ring, band_in_map);
+        const long long bytes = ring * row_bytes + dcnb::kBandStages * stage +
+                                dcnb::kBandStages * 16 + dcnb::kBandStages * dcnb::kBandDescInts * 4;
+        // one step's copies must fit in an mbarrier transaction count
+        if (bytes > kBandSmemLimit || band_in_map * row_bytes + stage >= (1 << 20)) continue;
+        a->x = x;
+        a->offset = offset;
+        a->mask = mask;
+        a->out = out;
+        a->H = H;
+        a->W = W;
+        a->C = C;
+        a->G = G;
+        a->kh = kh;
+        a->kw = kw;
+        a->K = K;
+        a->stride = stride;
+        a->pad = pad;
+        a->dil = dil;
+        a->Ho = Ho;
+        a->Wo = Wo;
+        a->rows_total = N * Ho;
+        a->th = th;
+        a->margin = margin;
+        a->ring_rows = (int)ring;
+        a->consumer_warps = warps;
+        a->runs_per_row = runs_per_row;
+        a->row_bytes = (uint32_t)row_bytes;
+        a->pix_bytes = (uint32_t)(C * es);
+        a->off_row_bytes = (uint32_t)off_row;
+        a->mask_row_bytes = (uint32_t)mask_row;
+        a->ring_bytes = (uint32_t)(ring * row_bytes);
+        a->stage_bytes = (uint32_t)stage;
+        a->div_G = make_div((uint32_t)G);
+        a->div_Ho = make_div((uint32_t)Ho);
+        a->div_runs = make_div((uint32_t)runs_per_row);
+        a->error = band_timeout_word();
+        *smem = (int)bytes;
+        *threads = 32 * (warps + 1);
+        return true;
+    }
+    return false;
+}
 
 template <typename T, int VB>
 const void* dcn_kernel_for(int softmax, int kh, int kw) {
@@ -36,10 +130,12 @@ const void* dcn_kernel_vb(int vb, int kh, int kw, int softmax) {
 
 extern "C" {
 
-int dcn_forward(const void* x, const void* offset, const void* mask, void* out, int N, int H,
-                int W, int C, int G, int kh, int kw, int stride, int pad, int dil,
-                int softmax_flag, int dtype, void* stream) {
+int dcn_forward_algo(const void* x, const void* offset, const void* mask, void* out, int N,
+                     int H, int W, int C, int G, int kh, int kw, int stride, int pad, int dil,
+                     int softmax_flag, int dtype, int algo, void* stream) {
     const int es = elem_bytes(dtype);
+    if (algo != DCN_ALGO_AUTO && algo != DCN_ALGO_GATHER && algo != DCN_ALGO_BAND)
+        return DCN_ERR_INVALID_ARG;
     if (es == 0 || N < 0 || H <= 0 || W <= 0 || C <= 0 || G <= 0 || C % G != 0 || kh <= 0 ||
         kw <= 0 || stride <= 0 || pad < 0 || dil <= 0 || (softmax_flag != 0 && softmax_flag != 1))
         return DCN_ERR_INVALID_ARG;
@@ -68,6 +164,19 @@ int dcn_forward(const void* x, const void* offset, const void* mask, void* out, 
     if (overlaps(out, o_bytes, x, x_bytes) || overlaps(out, o_bytes, offset, off_bytes) ||
         overlaps(out, o_bytes, mask, m_bytes))
         return DCN_ERR_INVALID_ARG;
+
+    if (algo != DCN_ALGO_GATHER) {
+        dcnb::BandArgs b;
+        int smem = 0, threads = 0;
+        if (band_config(x, offset, mask, out, N, H, W, C, G, kh, kw, stride, pad, dil, Ho, Wo,
+                        es, &b, &smem, &threads)) {
+            const void* fn = dtype == DCN_F16 ? band_kernel_for<__half>(softmax_flag, kh, kw)
+                                              : band_kernel_for<__nv_bfloat16>(softmax_flag, kh, kw);
+            // one CTA per SM, each a contiguous range of output rows
+            return launch(fn, b, b.rows_total, threads, smem, stream);
+        }
+        if (algo == DCN_ALGO_BAND) return DCN_ERR_UNSUPPORTED;
+    }
 
     const int vb = pick_vector_bytes(es, D, (uintptr_t)x | (uintptr_t)out);
     if (vb == 0) return DCN_ERR_MISALIGNED;
@@ -152,7 +261,12 @@ int dcn_forward(const void* x, const void* offset, const void* mask, void* out, 
     return launch(fn, a, a.num_tiles, 32 * warps, smem, stream);
 }
 
-// msda_forward and its reference-point variants: `sampling_loc` holds the
-// locations (ref_dim = 0) or the offsets (ref_dim = 2 / 4, with `ref` and
+int dcn_forward(const void* x, const void* offset, const void* mask, void* out, int N, int H,
+                int W, int C, int G, int kh, int kw, int stride, int pad, int dil,
+                int softmax_flag, int dtype, void* stream) {
+    return dcn_forward_algo(x, offset, mask, out, N, H, W, C, G, kh, kw, stride, pad, dil,
+                            softmax_flag, dtype, DCN_ALGO_AUTO, stream);
+}
+
 
 }  // extern "C"

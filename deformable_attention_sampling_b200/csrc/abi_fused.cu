@@ -1,11 +1,126 @@
-// C interface of libdcn_b200.so: dcnv4_fused_forward (the DCNv4 core fed by
-// its merged offset / mask linear).
+// C interface of libdcn_b200.so: dcnv4_fused_forward and
+// dcnv4_fused_forward_algo (the DCNv4 core fed by its merged offset / mask
+// linear).  Two kernels:
+//   - the band kernel with the linear on tcgen05 (dcn_band_fused.cuh): 16-bit
+//     data, 16 channels per group, C a multiple of 64 up to 256, 3 G K <= 256
+//     outputs, W <= 128, 16-byte aligned tensors and a band that fits in
+//     shared memory;
+//   - the gather kernel with the linear on warp-level mma.sync (dcn_fwd.cuh,
+//     FUSED): every other shape.
 #include "abi_common.cuh"
+#include "dcn_band_fused.cuh"
 #include "dcn_fwd.cuh"
 
 using namespace dcnb_abi;
 
 namespace {
+
+constexpr int kFusedSmemLimit = 227 * 1024;
+
+template <typename T>
+const void* band_fused_kernel_for(int kh, int kw) {
+    if (kh == 3 && kw == 3) return (const void*)dcnb::dcn_band_fused_kernel<T, 3>;
+    return (const void*)dcnb::dcn_band_fused_kernel<T, 0>;
+}
+
+// Launch configuration of the tcgen05 band kernel, or false when the shape or
+// the pointers do not qualify (or a tensor map cannot be made).
+bool band_fused_config(const void* x, const void* w_om, const void* b_om, void* out, int N,
+                       int H, int W, int C, int G, int kh, int kw, int pad, int dil, bool bf16,
+                       dcnb::BandFusedArgs* f, int* smem, int* threads) {
+    const int es = 2;
+    const int D = C / G;
+    const int K = kh * kw;
+    const int J = 3 * G * K;
+    if (D != 16 || C % 64 != 0 || C > 256 || J > 256 || W > 128) return false;
+    if ((((uintptr_t)x | (uintptr_t)w_om | (uintptr_t)out) % 16) != 0 ||
+        ((uintptr_t)b_om % es) != 0)
+        return false;
+    const int NJ = (J + 15) / 16 * 16;
+    const int kchunks = C / 64;
+    const long long row_bytes = (long long)W * C * es;
+    const int row_items = W * G;
+    const int runs_per_row = (row_items + 31) / 32;
+    const int consumer_warps = 16 - 2 - dcnb::kFusedEpilogueWarps;
+    const uint32_t a_bytes = (uint32_t)kchunks * 128u * 128u;
+    const uint32_t w_bytes = (uint32_t)kchunks * (uint32_t)NJ * 128u;
+    const uint32_t om_stride = (uint32_t)((J + 3) / 4 * 4);
+    uint32_t tmem_cols = 32;
+    while (tmem_cols < 2u * (uint32_t)NJ) tmem_cols <<= 1;
+    // the widest offset margin first (taps that leave the band are slow),
+    // then the most output rows per step
+    for (int margin = 6; margin >= 2; --margin) {
+        if (pad > margin + (kh - 1) * dil) break;
+        for (int th = std::min(4, std::min(128 / W, H)); th >= 1; --th) {
+            const uint32_t om_bytes = (uint32_t)((th * W * om_stride * 4 + 15) / 16 * 16);
+            const int band = dcnb::band_rows(th, 1, kh, dil, margin);
+            const int band_in_map = std::min(band, H);
+            long long ring = band + (long long)(dcnb::kBandStages - 1) * th;
+            ring = std::min(ring, 2LL * H);
+            ring = std::max<long long>(ring, band_in_map);
+            const long long bytes = 1024 + w_bytes + dcnb::kFusedStages * a_bytes +
+                                    ring * row_bytes + dcnb::kFusedStages * om_bytes +
+                                    (2 * dcnb::kBandStages + 4 * dcnb::kFusedStages + 1) * 8 +
+                                    dcnb::kBandStages * dcnb::kBandDescInts * 4 + 16 + NJ * 4;
+            const long long tx = band_in_map * row_bytes + (long long)kchunks * th * W * 128;
+            if (bytes > kFusedSmemLimit || tx >= (1 << 20)) continue;
+            dcnb::BandArgs& a = f->b;
+            a.x = x;
+            a.offset = nullptr;
+            a.mask = nullptr;
+            a.out = out;
+            a.H = H;
+            a.W = W;
+            a.C = C;
+            a.G = G;
+            a.kh = kh;
+            a.kw = kw;
+            a.K = K;
+            a.stride = 1;
+            a.pad = pad;
+            a.dil = dil;
+            a.Ho = H;
+            a.Wo = W;
+            a.rows_total = N * H;
+            a.th = th;
+            a.margin = margin;
+            a.ring_rows = (int)ring;
+            a.consumer_warps = consumer_warps;
+            a.runs_per_row = runs_per_row;
+            a.row_bytes = (uint32_t)row_bytes;
+            a.pix_bytes = (uint32_t)(C * es);
+            a.off_row_bytes = 0;
+            a.mask_row_bytes = 0;
+            a.ring_bytes = (uint32_t)(ring * row_bytes);
+            a.stage_bytes = 0;
+            a.div_G = make_div((uint32_t)G);
+            a.div_Ho = make_div((uint32_t)H);
+            a.div_runs = make_div((uint32_t)runs_per_row);
+            a.error = nullptr;
+            f->b_om = b_om;
+            f->J = J;
+            f->NJ = NJ;
+            f->kchunks = kchunks;
+            f->a_rows = th * W;
+            f->consumer_warps = consumer_warps;
+            f->tmem_cols = tmem_cols;
+            f->a_bytes = a_bytes;
+            f->a_box_bytes = (uint32_t)kchunks * (uint32_t)(th * W) * 128u;
+            f->w_bytes = w_bytes;
+            f->om_stride = om_stride;
+            f->om_bytes = om_bytes;
+            if (!encode_tmap_2d(&f->tmap_x, x, bf16, (uint64_t)C, (uint64_t)N * H * W,
+                                (uint64_t)C * es, 64, (uint32_t)(th * W)) ||
+                !encode_tmap_2d(&f->tmap_w, w_om, bf16, (uint64_t)C, (uint64_t)J,
+                                (uint64_t)C * es, 64, (uint32_t)NJ))
+                return false;
+            *smem = (int)bytes;
+            *threads = 32 * (consumer_warps + 2 + dcnb::kFusedEpilogueWarps);
+            return true;
+        }
+    }
+    return false;
+}
 
 template <typename T, int VB>
 const void* dcn_fused_kernel_for(int kh, int kw) {
@@ -30,10 +145,12 @@ const void* dcn_fused_kernel_vb(int vb, int kh, int kw) {
 
 extern "C" {
 
-int dcnv4_fused_forward(const void* x, const void* w_om, const void* b_om, void* out, int N,
-                        int H, int W, int C, int G, int kh, int kw, int pad, int dil, int dtype,
-                        void* stream) {
+int dcnv4_fused_forward_algo(const void* x, const void* w_om, const void* b_om, void* out,
+                             int N, int H, int W, int C, int G, int kh, int kw, int pad, int dil,
+                             int dtype, int algo, void* stream) {
     const int es = elem_bytes(dtype);
+    if (algo != DCN_ALGO_AUTO && algo != DCN_ALGO_GATHER && algo != DCN_ALGO_BAND)
+        return DCN_ERR_INVALID_ARG;
     if (es == 0 || N < 0 || H <= 0 || W <= 0 || C <= 0 || G <= 0 || C % G != 0 || kh <= 0 ||
         kw <= 0 || pad < 0 || dil <= 0)
         return DCN_ERR_INVALID_ARG;
@@ -60,6 +177,20 @@ int dcnv4_fused_forward(const void* x, const void* w_om, const void* b_om, void*
     if (overlaps(out, xb, x, xb) || overlaps(out, xb, w_om, (long long)J * C * es) ||
         (b_om && overlaps(out, xb, b_om, (long long)J * es)))
         return DCN_ERR_INVALID_ARG;
+
+    if (algo != DCN_ALGO_GATHER) {
+        dcnb::BandFusedArgs f;
+        int smem = 0, threads = 0;
+        if (band_fused_config(x, w_om, b_om, out, N, H, W, C, G, kh, kw, pad, dil,
+                              dtype == DCN_BF16, &f, &smem, &threads)) {
+            f.b.error = band_timeout_word();
+            const void* fn = dtype == DCN_F16 ? band_fused_kernel_for<__half>(kh, kw)
+                                              : band_fused_kernel_for<__nv_bfloat16>(kh, kw);
+            // one CTA per SM (the shared-memory footprint allows no more)
+            return launch(fn, f, f.b.rows_total, threads, smem, stream);
+        }
+        if (algo == DCN_ALGO_BAND) return DCN_ERR_UNSUPPORTED;
+    }
 
     const int vb = pick_vector_bytes(es, D, (uintptr_t)x | (uintptr_t)out);
     if (vb == 0) return DCN_ERR_MISALIGNED;
@@ -141,6 +272,13 @@ int dcnv4_fused_forward(const void* x, const void* w_om, const void* b_om, void*
     }
     if (!fn) return DCN_ERR_UNSUPPORTED;
     return launch(fn, a, a.num_tiles, 32 * warps, smem, stream);
+}
+
+int dcnv4_fused_forward(const void* x, const void* w_om, const void* b_om, void* out, int N,
+                        int H, int W, int C, int G, int kh, int kw, int pad, int dil, int dtype,
+                        void* stream) {
+    return dcnv4_fused_forward_algo(x, w_om, b_om, out, N, H, W, C, G, kh, kw, pad, dil, dtype,
+                                    DCN_ALGO_AUTO, stream);
 }
 
 }  // extern "C"

@@ -91,6 +91,46 @@ DCN_API int dcn_forward(const void* x, const void* offset, const void* mask, voi
                 void* stream);
 
 /*
+ * dcn_forward_algo - dcn_forward with a choice of kernel.
+ *
+ * The same operator, arguments, layouts, limits and errors as dcn_forward
+ * (which is dcn_forward_algo with DCN_ALGO_AUTO); `algo` picks the kernel:
+ *   DCN_ALGO_GATHER  corners read through the L1 cache; every shape;
+ *   DCN_ALGO_BAND    the input rows a CTA's output rows can reach (window plus
+ *                    a margin of up to 6 rows for the offsets) staged in shared
+ *                    memory by bulk copies, corners read from there (taps whose
+ *                    offsets leave the band read global memory); only for
+ *                    16-bit data with 16 channels per group, C * 2 a multiple
+ *                    of 128 bytes, all four tensors 16-byte aligned, offset and
+ *                    mask rows of a multiple of 16 bytes and a band that fits in
+ *                    shared memory (W * C * 2 bytes per row): DCN_ERR_UNSUPPORTED
+ *                    otherwise;
+ *   DCN_ALGO_AUTO    the band kernel where it applies, else the gather kernel.
+ * The two kernels round the same float32 sums; their outputs may differ in the
+ * last bit where the order of the float32 additions differs.
+ * Errors: as dcn_forward, plus DCN_ERR_INVALID_ARG for an unknown `algo`.
+ */
+typedef enum { DCN_ALGO_AUTO = 0, DCN_ALGO_GATHER = 1, DCN_ALGO_BAND = 2 } dcn_algo_t;
+
+DCN_API int dcn_forward_algo(const void* x, const void* offset, const void* mask, void* out,
+                     int N, int H, int W, int C, int G, int kh, int kw,
+                     int stride, int pad, int dil, int softmax_flag, int dtype,
+                     int algo, void* stream);
+
+/*
+ * dcn_forward_timeouts - bounded waits of the band kernel that ran out.
+ *
+ * Every wait of the band kernel on its pipeline barriers gives up after about
+ * two seconds; one that does sets a word on the current device, and its CTA
+ * stops (the output of that call is then incomplete).  This returns that
+ * word (0: no wait has ever run out on this device since the library was
+ * loaded), reading it with a synchronous copy: it waits for the device's
+ * preceding work.  No counterpart on the pages: a guard of this library's
+ * own pipeline.  Returns DCN_ERR_CUDA if the read fails.
+ */
+DCN_API int dcn_forward_timeouts(void);
+
+/*
  * msda_forward - multi-scale deformable attention core, forward.
  *
  * Defined by "Deformable DETR: Learn Where to Read", "A learned location can
@@ -155,6 +195,31 @@ DCN_API int msda_forward(const void* value, const int64_t* spatial_shapes,
 DCN_API int dcnv4_fused_forward(const void* x, const void* w_om, const void* b_om, void* out,
                  int N, int H, int W, int C, int G, int kh, int kw, int pad, int dil,
                  int dtype, void* stream);
+
+/*
+ * dcnv4_fused_forward_algo - dcnv4_fused_forward with a choice of kernel.
+ *
+ * The same operator, arguments, layouts and errors as dcnv4_fused_forward
+ * (which is this call with DCN_ALGO_AUTO); `algo` picks the kernel:
+ *   DCN_ALGO_GATHER  corners read through L1, the linear per warp run on the
+ *                    warp-level tensor-core path (mma.sync);
+ *   DCN_ALGO_BAND    input rows staged in shared memory (as dcn_forward_algo's
+ *                    band kernel) and the linear of each step's pixels (up to
+ *                    128) as one tcgen05 product (M = 128, N = 3GK rounded up to
+ *                    16, K = C) with float32 accumulators in tensor memory, fed
+ *                    by tensor-map loads; only for 16 channels per group, C a
+ *                    multiple of 64 up to 256, 3 G K <= 256, W <= 128 and
+ *                    16-byte aligned x, w_om and out: DCN_ERR_UNSUPPORTED
+ *                    otherwise;
+ *   DCN_ALGO_AUTO    the band kernel where it applies, else the gather kernel.
+ * Both keep the offsets and masks in float32 on chip; the two products add in
+ * different orders, so outputs may differ in the last bits.
+ * Errors: as dcnv4_fused_forward, plus DCN_ERR_INVALID_ARG for an unknown
+ * `algo`.
+ */
+DCN_API int dcnv4_fused_forward_algo(const void* x, const void* w_om, const void* b_om,
+                 void* out, int N, int H, int W, int C, int G, int kh, int kw, int pad,
+                 int dil, int dtype, int algo, void* stream);
 
 /*
  * msda_forward_points - msda_forward fed from reference points or boxes.

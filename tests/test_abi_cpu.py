@@ -103,6 +103,36 @@ def test_dcn_forward_validation(lib, change, status):
     assert dcnb.dcn_launch_count() == before
 
 
+def call_dcn_algo(lib, algo, **kw):
+    args = dict(x=X, offset=OFF, mask=MASK, out=OUT, N=2, H=8, W=8, C=64, G=4, kh=3, kw=3,
+                stride=1, pad=1, dil=1, softmax_flag=0, dtype=F16, stream=None)
+    args.update(kw)
+    return lib.dcn_forward_algo(args["x"], args["offset"], args["mask"], args["out"],
+                                args["N"], args["H"], args["W"], args["C"], args["G"],
+                                args["kh"], args["kw"], args["stride"], args["pad"],
+                                args["dil"], args["softmax_flag"], args["dtype"], algo,
+                                args["stream"])
+
+
+@pytest.mark.parametrize("algo,change,status", [
+    (3, {}, dcnb.DCN_ERR_INVALID_ARG),                           # unknown algo
+    (-1, {}, dcnb.DCN_ERR_INVALID_ARG),
+    (dcnb.DCN_ALGO_BAND, dict(dtype=0), dcnb.DCN_ERR_UNSUPPORTED),           # float32
+    (dcnb.DCN_ALGO_BAND, dict(C=32, G=1), dcnb.DCN_ERR_UNSUPPORTED),         # D = 32
+    (dcnb.DCN_ALGO_BAND, dict(C=48, G=3), dcnb.DCN_ERR_UNSUPPORTED),         # 96-byte pixels
+    (dcnb.DCN_ALGO_BAND, dict(x=X + 8), dcnb.DCN_ERR_UNSUPPORTED),           # not 16-byte aligned
+    (dcnb.DCN_ALGO_BAND, dict(W=7), dcnb.DCN_ERR_UNSUPPORTED),               # mask rows of 504 bytes
+    (dcnb.DCN_ALGO_BAND, dict(W=4000), dcnb.DCN_ERR_UNSUPPORTED),            # a band of 500 KB rows
+    (dcnb.DCN_ALGO_BAND, dict(pad=9, H=30, W=30), dcnb.DCN_ERR_UNSUPPORTED),  # bands outside the map
+    (dcnb.DCN_ALGO_GATHER, dict(C=15), dcnb.DCN_ERR_INVALID_ARG),            # the common checks
+    (dcnb.DCN_ALGO_BAND, dict(N=0), dcnb.DCN_OK),
+])
+def test_dcn_forward_algo_validation(lib, algo, change, status):
+    before = dcnb.dcn_launch_count()
+    assert call_dcn_algo(lib, algo, **change) == status
+    assert dcnb.dcn_launch_count() == before
+
+
 def call_msda(lib, **kw):
     args = dict(value=X, shapes=OFF, starts=OFF + 1024, loc=MASK, attn=MASK + 2 ** 24, out=OUT,
                 N=2, Lq=100, M=8, D=32, L=4, K=4, dtype=0, stream=None)

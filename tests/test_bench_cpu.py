@@ -44,7 +44,7 @@ def test_gpus_flag_never_silently_runs_one_rank(bench):
     import sys
     import torch
     args = argparse.Namespace(gpus=2, steps=3, warmup=3, impl="b200",
-                              workload="dcnv3_f32_1x14x14x64_g4", pass_="forward")
+                              workload="dcnv3_f32_1x14x14x64_g4", pass_="forward", algo="auto")
     cmd = bench.torchrun_command(args, 29511)
     assert "--nproc-per-node=2" in cmd and "--master-addr=127.0.0.1" in cmd
     assert cmd[cmd.index("--gpus") + 1] == "2"

@@ -1,6 +1,10 @@
 """GPU parity of dcnv4_fused_forward (the DCNv4 core fed by its merged
-offset / mask linear, computed per warp on the tensor cores) against the
-float64 oracle: the merged linear as a float64 matmul, then the DCN oracle."""
+offset / mask linear on the tensor cores) against the float64 oracle: the
+merged linear as a float64 matmul, then the DCN oracle.
+
+Both kernels are checked: the band kernel with the linear as one tcgen05
+product per step ("band"), and the gather kernel with the linear per warp run
+on mma.sync ("gather"); "auto" takes the band kernel where it applies."""
 import numpy as np
 import pytest
 import torch
@@ -14,10 +18,10 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def run(inp, w, bias=True):
+def run(inp, w, bias=True, algo="auto"):
     d = {k: v.to(DEV) for k, v in inp.items()}
     out = dcnb.dcnv4_fused(d["x"], d["w_om"], d["b_om"] if bias else None, groups=w.G, kh=w.kh,
-                           kw=w.kw, pad=w.pad, dil=w.dil)
+                           kw=w.kw, pad=w.pad, dil=w.dil, algo=algo)
     torch.cuda.synchronize()
     return out
 
@@ -29,12 +33,13 @@ def ref(inp, w, n=None, bias=True):
     return out
 
 
-def test_fused_headline_shape_full_size():
+@pytest.mark.parametrize("algo", ["band", "gather"])
+def test_fused_headline_shape_full_size(algo):
     w = gen.WORKLOADS["dcnv4_fused_f16_64x56x56x64_g4"]
     inp = gen.front_end_inputs(w, seed=0)
-    out = run(inp, w)
-    for n in (0, w.N - 1):
-        compare(out[n:n + 1], ref(inp, w, n), f"{w.name} image {n}")
+    out = run(inp, w, algo=algo)
+    for n in (0, w.N // 2, w.N - 1):
+        compare(out[n:n + 1], ref(inp, w, n), f"{w.name} {algo} image {n}")
 
 
 CASES = [
@@ -55,6 +60,44 @@ def test_fused_small_shapes(case):
     w = gen.FusedWorkload("small", N=N, H=H, W=W, C=C, G=G, kh=k, kw=k, pad=pad, dil=dil, dtype=dt)
     inp = gen.front_end_inputs(w, seed=4)
     compare(run(inp, w), ref(inp, w), str(case))
+
+
+BAND_CASES = [
+    # N, H, W, C, G, k, pad, dil, dtype
+    (2, 12, 14, 64, 4, 3, 1, 1, "f16"),
+    (2, 10, 20, 128, 8, 3, 1, 1, "bf16"),    # two 64-channel K slices, 216 outputs
+    (1, 9, 128, 64, 4, 3, 1, 1, "f16"),      # 128 pixels per step: the whole M tile
+    (3, 5, 9, 64, 4, 1, 0, 1, "bf16"),       # 1 x 1 window: 12 outputs
+    (2, 12, 16, 64, 4, 3, 2, 2, "f16"),      # dilation 2
+    (5, 3, 8, 64, 4, 3, 1, 1, "f16"),        # several images per CTA
+    (1, 30, 40, 256, 16, 1, 0, 1, "bf16"),   # C = 256: four K slices
+]
+
+
+@pytest.mark.parametrize("case", BAND_CASES, ids=[f"band{i}" for i in range(len(BAND_CASES))])
+def test_fused_band_kernel_small_shapes(case):
+    N, H, W, C, G, k, pad, dil, dt = case
+    w = gen.FusedWorkload("band", N=N, H=H, W=W, C=C, G=G, kh=k, kw=k, pad=pad, dil=dil,
+                          dtype=dt)
+    inp = gen.front_end_inputs(w, seed=6)
+    expect = ref(inp, w)
+    band = run(inp, w, algo="band")
+    compare(band, expect, f"{case} band")
+    compare(run(inp, w, algo="gather"), expect, f"{case} gather")
+    assert torch.equal(run(inp, w, algo="auto"), band)
+
+
+def test_fused_band_kernel_rejects_other_shapes():
+    w = gen.FusedWorkload("no", N=1, H=6, W=7, C=32, G=2, dtype="f16")   # C not a multiple of 64
+    inp = gen.front_end_inputs(w, seed=6)
+    with pytest.raises(dcnb.DcnError) as e:
+        run(inp, w, algo="band")
+    assert e.value.status == dcnb.DCN_ERR_UNSUPPORTED
+    compare(run(inp, w, algo="auto"), ref(inp, w), "auto falls back")
+
+
+def test_fused_no_wait_ran_out():
+    assert dcnb.dcn_forward_timeouts() == 0
 
 
 def test_fused_without_bias_and_one_launch():
