@@ -20,6 +20,11 @@ constexpr int kBandMarginRows = 6;     // offset margin of the band, at most
 constexpr int kBandMinMarginRows = 2;
 constexpr int kBandSmemLimit = 227 * 1024;
 constexpr int kBandTargetItems = 14 * 32;   // items per step
+#ifndef DCN_BAND_STAGES
+#define DCN_BAND_STAGES 2
+#endif
+constexpr int kBandStepsInFlight = DCN_BAND_STAGES;   // 2 .. dcnb::kBandMaxStages
+static_assert(kBandStepsInFlight >= 2 && kBandStepsInFlight <= dcnb::kBandMaxStages, "stages");
 
 template <typename T>
 const void* band_kernel_for(int softmax, int kh, int kw) {
@@ -46,7 +51,8 @@ bool band_config(const void* x, const void* offset, const void* mask, void* out,
     const long long mask_row = (long long)Wo * G * K * es;
     if (off_row % 16 != 0 || mask_row % 16 != 0) return false;
     const long long row_items = (long long)Wo * G;
-    const int runs_per_row = (int)((row_items + 31) / 32);
+    const int run_items = 32 / dcnb::kBandLanesPerItem;
+    const int runs_per_row = (int)((row_items + run_items - 1) / run_items);
     int th = (int)((kBandTargetItems + row_items - 1) / row_items);
     th = std::max(1, std::min(th, std::min(4, Ho)));
     const int warps = std::min(dcnb::kBandMaxConsumerWarps, th * runs_per_row);
@@ -55,11 +61,12 @@ bool band_config(const void* x, const void* offset, const void* mask, void* out,
         if (pad > margin + (kh - 1) * dil) break;   // every band must meet the map
         const int band = dcnb::band_rows(th, stride, kh, dil, margin);
         const int band_in_map = std::min(band, H);
-        long long ring = band + (long long)(dcnb::kBandStages - 1) * th * stride;
+        long long ring = band + (long long)(kBandStepsInFlight - 1) * th * stride;
         ring = std::min(ring, 2LL * H);
         ring = std::max<long long>(ring, band_in_map);
-        const long long bytes = ring * row_bytes + dcnb::kBandStages * stage +
-                                dcnb::kBandStages * 16 + dcnb::kBandStages * dcnb::kBandDescInts * 4;
+        const long long bytes = ring * row_bytes + kBandStepsInFlight * stage +
+                                kBandStepsInFlight * 16 +
+                                kBandStepsInFlight * dcnb::kBandDescInts * 4;
         // one step's copies must fit in an mbarrier transaction count
         if (bytes > kBandSmemLimit || band_in_map * row_bytes + stage >= (1 << 20)) continue;
         a->x = x;
@@ -83,6 +90,7 @@ bool band_config(const void* x, const void* offset, const void* mask, void* out,
         a->margin = margin;
         a->ring_rows = (int)ring;
         a->consumer_warps = warps;
+        a->stages = kBandStepsInFlight;
         a->runs_per_row = runs_per_row;
         a->row_bytes = (uint32_t)row_bytes;
         a->pix_bytes = (uint32_t)(C * es);

@@ -16,6 +16,7 @@ using namespace dcnb_abi;
 namespace {
 
 constexpr int kFusedSmemLimit = 227 * 1024;
+constexpr int kFusedMaxStages = 3;
 
 template <typename T>
 const void* band_fused_kernel_for(int kh, int kw) {
@@ -40,30 +41,43 @@ bool band_fused_config(const void* x, const void* w_om, const void* b_om, void* 
     const int kchunks = C / 64;
     const long long row_bytes = (long long)W * C * es;
     const int row_items = W * G;
-    const int runs_per_row = (row_items + 31) / 32;
+    const int run_items = 32 / dcnb::kBandLanesPerItem;
+    const int runs_per_row = (row_items + run_items - 1) / run_items;
     const int consumer_warps = 16 - 2 - dcnb::kFusedEpilogueWarps;
-    const uint32_t a_bytes = (uint32_t)kchunks * 128u * 128u;
     const uint32_t w_bytes = (uint32_t)kchunks * (uint32_t)NJ * 128u;
     const uint32_t om_stride = (uint32_t)((J + 3) / 4 * 4);
-    uint32_t tmem_cols = 32;
-    while (tmem_cols < 2u * (uint32_t)NJ) tmem_cols <<= 1;
-    // the widest offset margin first (taps that leave the band are slow),
-    // then the most output rows per step
-    for (int margin = 6; margin >= 2; --margin) {
-        if (pad > margin + (kh - 1) * dil) break;
-        for (int th = std::min(4, std::min(128 / W, H)); th >= 1; --th) {
+    // candidates in order of preference: offset margin (taps that leave the
+    // band are slow) and steps in flight (the product's result must be ready
+    // before the samplers reach its step), then the most output rows per step
+    static const int kPlans[][2] = {{6, 3}, {5, 3}, {6, 2}, {5, 2}, {4, 3}, {4, 2},
+                                    {3, 3}, {3, 2}, {2, 3}, {2, 2}};
+    for (const auto& plan : kPlans) {
+        const int margin = plan[0], ns = plan[1];
+        if (pad > margin + (kh - 1) * dil) continue;
+        {
+            if (ns > kFusedMaxStages || (uint32_t)ns * (uint32_t)NJ > 512u) continue;
+            for (int th = std::min(4, std::min(128 / W, H)); th >= 1; --th) {
+            // A stage: the step's th * W pixel rows, rounded to 64 or 128 (the
+            // product reads 128 rows; rows past the tile only reach accumulator
+            // lanes that are never read)
+            const int a_rows_alloc = th * W <= 64 ? 64 : 128;
+            const uint32_t a_bytes = (uint32_t)kchunks * (uint32_t)a_rows_alloc * 128u;
             const uint32_t om_bytes = (uint32_t)((th * W * om_stride * 4 + 15) / 16 * 16);
             const int band = dcnb::band_rows(th, 1, kh, dil, margin);
             const int band_in_map = std::min(band, H);
-            long long ring = band + (long long)(dcnb::kBandStages - 1) * th;
+            long long ring = band + (long long)(ns - 1) * th;
             ring = std::min(ring, 2LL * H);
             ring = std::max<long long>(ring, band_in_map);
-            const long long bytes = 1024 + w_bytes + dcnb::kFusedStages * a_bytes +
-                                    ring * row_bytes + dcnb::kFusedStages * om_bytes +
-                                    (2 * dcnb::kBandStages + 4 * dcnb::kFusedStages + 1) * 8 +
-                                    dcnb::kBandStages * dcnb::kBandDescInts * 4 + 16 + NJ * 4;
+            // 1 KB of alignment slack, tiles, ring, om buffers, barriers
+            // (2 per step in flight for the ring and 4 for the product, plus
+            // the weight tile's), descriptors, the TMEM address and the bias
+            const long long bytes = 1024 + w_bytes + (long long)ns * a_bytes + ring * row_bytes +
+                                    (long long)ns * om_bytes + (6LL * ns + 1) * 8 +
+                                    (long long)ns * dcnb::kBandDescInts * 4 + 16 + NJ * 4;
             const long long tx = band_in_map * row_bytes + (long long)kchunks * th * W * 128;
             if (bytes > kFusedSmemLimit || tx >= (1 << 20)) continue;
+            uint32_t tmem_cols = 32;
+            while (tmem_cols < (uint32_t)(ns * NJ)) tmem_cols <<= 1;
             dcnb::BandArgs& a = f->b;
             a.x = x;
             a.offset = nullptr;
@@ -86,6 +100,7 @@ bool band_fused_config(const void* x, const void* w_om, const void* b_om, void* 
             a.margin = margin;
             a.ring_rows = (int)ring;
             a.consumer_warps = consumer_warps;
+            a.stages = ns;
             a.runs_per_row = runs_per_row;
             a.row_bytes = (uint32_t)row_bytes;
             a.pix_bytes = (uint32_t)(C * es);
@@ -117,6 +132,7 @@ bool band_fused_config(const void* x, const void* w_om, const void* b_om, void* 
             *smem = (int)bytes;
             *threads = 32 * (consumer_warps + 2 + dcnb::kFusedEpilogueWarps);
             return true;
+            }
         }
     }
     return false;

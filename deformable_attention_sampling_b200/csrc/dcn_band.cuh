@@ -51,8 +51,26 @@
 
 namespace dcnb {
 
-constexpr int kBandStages = 2;            // stage buffers (offsets, masks, descriptor)
-constexpr int kBandMaxConsumerWarps = 15;   // with the producer: 16 warps, 128 registers each
+// Steps in flight (stage buffers of offsets and masks, descriptors, barrier
+// pairs): a launch parameter between 2 and kBandMaxStages.
+constexpr int kBandMaxStages = 4;
+// Lanes per (pixel, group) item of the band samplers: 1 (each lane reads both
+// 16-byte halves of the group, 16 channels) or 2 (one half each).  Sampler
+// warps per CTA, with the producer warp: 16 warps of up to 128 registers at
+// one lane per item, 25 warps of up to 72 registers at two.
+#ifndef DCN_BAND_LPI
+#define DCN_BAND_LPI 1
+#endif
+constexpr int kBandLanesPerItem = DCN_BAND_LPI;
+static_assert(kBandLanesPerItem == 1 || kBandLanesPerItem == 2, "1 or 2 lanes per item");
+// Tap geometry computed one (1) or two (2) taps ahead of the accumulation.
+#ifndef DCN_BAND_AHEAD
+#define DCN_BAND_AHEAD 1
+#endif
+#ifndef DCN_BAND_WARPS
+#define DCN_BAND_WARPS (DCN_BAND_LPI == 1 ? 15 : 24)
+#endif
+constexpr int kBandMaxConsumerWarps = DCN_BAND_WARPS;
 constexpr int kBandMaxThreads = 32 * (kBandMaxConsumerWarps + 1);
 constexpr int kBandDescInts = 8;
 constexpr unsigned long long kBandWaitNs = 2000000000ull;   // bound of every wait
@@ -75,7 +93,8 @@ struct BandArgs {
     int margin;               // offset margin of the band, rows above and below
     int ring_rows;            // rows in the ring
     int consumer_warps;       // warps that sample; one more warp produces
-    int runs_per_row;         // ceil(Wo * G / 32)
+    int stages;               // steps in flight: stage buffers, descriptors, barrier pairs
+    int runs_per_row;         // ceil(Wo * G / items per warp run)
     uint32_t row_bytes;       // W * C * 2: one input row
     uint32_t pix_bytes;       // C * 2
     uint32_t off_row_bytes;   // Wo * G * K * 2 * 2: offsets of one output row
@@ -162,6 +181,34 @@ __device__ __forceinline__ void lds128(uint32_t addr, uint32_t* w) {
                  : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr));
 }
 
+// An (x, y) offset pair and one modulation of type OT from shared memory
+// (32-bit shared addresses), widened to float32.  Volatile for the same reason
+// as lds128.
+template <typename OT>
+__device__ __forceinline__ void lds_pair(uint32_t addr, float& x, float& y) {
+    if constexpr (sizeof(OT) == 4) {
+        asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(x), "=f"(y) : "r"(addr));
+    } else {
+        uint32_t w;
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w) : "r"(addr));
+        x = Elem<OT>::lo(w);
+        y = Elem<OT>::hi(w);
+    }
+}
+
+template <typename OT>
+__device__ __forceinline__ float lds_one(uint32_t addr) {
+    if constexpr (sizeof(OT) == 4) {
+        float v;
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+        return v;
+    } else {
+        unsigned short h;
+        asm volatile("ld.shared.b16 %0, [%1];" : "=h"(h) : "r"(addr));
+        return Elem<OT>::lo((uint32_t)h);
+    }
+}
+
 // ------------------------------------------------------------- steps -------
 
 // The step that starts at flat output row `cur` (< end): image n, first row o,
@@ -187,40 +234,57 @@ struct BandDesc {
 // One (pixel, group) item of a band step, sampled by one lane: the item's
 // taps read their corners from the staged band (or, for taps that leave it,
 // from global memory), accumulate in float32 and store the item's 16 outputs.
-// offp / maskp: the item's K offset pairs and K modulations (or logits) in
-// shared memory, as T (staged from the tensors) or float (computed in-kernel).
+// off_s / mask_s: shared addresses of the item's K offset pairs and K
+// modulations (or logits), as T (staged from the tensors) or float (computed
+// in-kernel).
 // Lanes with active = false compute but store nothing.
-template <typename T, typename OT, bool SOFTMAX, int KF>
+template <typename T, typename OT, bool SOFTMAX, int KF, int LPI>
 __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc,
                                           uint32_t ring_s, int n, int oy, int item, bool active,
-                                          const OT* offp, const OT* maskp, int lane) {
+                                          uint32_t off_s, uint32_t mask_s, int lane) {
+    constexpr uint32_t OB = sizeof(OT);
     constexpr int UNROLL = KF ? KF * KF : 1;
+    constexpr int NH = 2 / LPI;            // 16-byte halves of the group per lane
     const int kh = KF ? KF : a.kh;
     const int kw = KF ? KF : a.kw;
     const int K = kh * kw;
     const int row_items = a.Wo * a.G;
-    const int rot = (lane >> 2) & 1;
     const int ox = (int)a.div_G.div((uint32_t)item);
     const int g = item - ox * a.G;
     const int bx = ox * a.stride - a.pad;
     const int by = oy * a.stride - a.pad;
-    const uint32_t lane_b0 = (uint32_t)(g * 32 + rot * 16);
-    const uint32_t lane_b1 = (uint32_t)(g * 32 + (rot ^ 1) * 16);
+    // byte offsets, inside the group's 32 bytes, of the halves this lane reads
+    // in order: one lane per item reads both, lanes 4-7 of every eight in the
+    // opposite order; two lanes per item read one half each
+    uint32_t hb[NH];
+    if constexpr (LPI == 1) {
+        const int rot = (lane >> 2) & 1;
+        hb[0] = (uint32_t)(rot * 16);
+        hb[NH - 1] = (uint32_t)((rot ^ 1) * 16);
+    } else {
+        hb[0] = (uint32_t)((lane & 1) * 16);
+    }
+    // shared address of this lane's first half in ring slot 0, pixel 0, and
+    // the step from the first half to the second
+    const uint32_t lane_s = ring_s + (uint32_t)(g * 32) + hb[0];
+    const uint32_t dh = hb[NH - 1] - hb[0];
+    const int span = dsc.y_hi - dsc.y_lo;
+    const int slot_lo = dsc.slot_lo;
     const char* xg = static_cast<const char*>(a.x) +
                      (long long)n * a.H * a.row_bytes + g * 32;
 
     float zmax = 0.f, inv_sum = 1.f;
     if constexpr (SOFTMAX) {
-        zmax = Elem<OT>::one(maskp);
-        for (int k = 1; k < K; ++k) zmax = fmaxf(zmax, Elem<OT>::one(maskp + k));
+        zmax = lds_one<OT>(mask_s);
+        for (int k = 1; k < K; ++k) zmax = fmaxf(zmax, lds_one<OT>(mask_s + k * OB));
         float s = 0.f;
-        for (int k = 0; k < K; ++k) s += expf(Elem<OT>::one(maskp + k) - zmax);
+        for (int k = 0; k < K; ++k) s += expf(lds_one<OT>(mask_s + k * OB) - zmax);
         inv_sum = 1.f / s;
     }
 
-    float acc[16];
+    float acc[8 * NH];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 8 * NH; ++i) acc[i] = 0.f;
 
     // Tap geometry: corner weights (zero outside the map, m folded in),
     // shared addresses of the four corners' halves, and whether a row
@@ -236,8 +300,8 @@ __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc
     auto geometry = [&]() {
         const int k = nix * kh + niy;
         float dx, dy;
-        load_pair<OT>(offp + 2 * k, dx, dy);
-        float m = Elem<OT>::one(maskp + k);
+        lds_pair<OT>(off_s + 2 * k * OB, dx, dy);
+        float m = lds_one<OT>(mask_s + k * OB);
         if constexpr (SOFTMAX) m = expf(m - zmax) * inv_sum;
         Tap t;
         float fx = floorf(dx), fy = floorf(dy);
@@ -254,20 +318,22 @@ __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc
         t.w[1] = wx1 * wy0;
         t.w[2] = wx0 * wy1;
         t.w[3] = wx1 * wy1;
-        const bool in0 = y0 >= dsc.y_lo && y0 <= dsc.y_hi;
-        const bool in1 = y0 + 1 >= dsc.y_lo && y0 + 1 <= dsc.y_hi;
+        // rows relative to the band; a row inside the map but outside the
+        // band sends the tap to global memory
+        const int r0 = y0 - dsc.y_lo;
+        const bool in0 = (unsigned)r0 <= (unsigned)span;
+        const bool in1 = (unsigned)(r0 + 1) <= (unsigned)span;
         t.fb = (vy0 && !in0) || (vy1 && !in1);
         // rows clamped into the band, columns into the map: every
         // shared read is of a staged row
-        const int r0 = min(max(y0, dsc.y_lo), dsc.y_hi) - dsc.y_lo;
-        const int r1 = min(max(y0 + 1, dsc.y_lo), dsc.y_hi) - dsc.y_lo;
-        int s0 = dsc.slot_lo + r0, s1 = dsc.slot_lo + r1;
+        int s0 = slot_lo + min(max(r0, 0), span);
+        int s1 = slot_lo + min(max(r0 + 1, 0), span);
         if (s0 >= a.ring_rows) s0 -= a.ring_rows;
         if (s1 >= a.ring_rows) s1 -= a.ring_rows;
         const uint32_t c0 = (uint32_t)(vx0 ? x0 : 0) * a.pix_bytes;
         const uint32_t c1 = (uint32_t)(vx1 ? x0 + 1 : 0) * a.pix_bytes;
-        const uint32_t b0 = ring_s + (uint32_t)s0 * a.row_bytes;
-        const uint32_t b1 = ring_s + (uint32_t)s1 * a.row_bytes;
+        const uint32_t b0 = lane_s + (uint32_t)s0 * a.row_bytes;
+        const uint32_t b1 = lane_s + (uint32_t)s1 * a.row_bytes;
         t.s[0] = b0 + c0;
         t.s[1] = b0 + c1;
         t.s[2] = b1 + c0;
@@ -282,10 +348,10 @@ __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc
     };
     // the four corners of tap t into v (shared memory, then the global
     // fallback for lanes whose tap leaves the band)
-    uint32_t v[4][8];
+    uint32_t v[4][4 * NH];
     auto load_shared = [&](const Tap& t, int c) {
-        lds128(t.s[c] + lane_b0, &v[c][0]);
-        lds128(t.s[c] + lane_b1, &v[c][4]);
+#pragma unroll
+        for (int h = 0; h < NH; ++h) lds128(h ? t.s[c] + dh : t.s[c], &v[c][4 * h]);
     };
     auto load_fallback = [&](const Tap& t) {
         if (__any_sync(0xffffffffu, t.fb) && t.fb) {
@@ -299,10 +365,9 @@ __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc
             const long long r1 = (long long)(vy1 ? t.y0 + 1 : 0) * a.row_bytes;
             const long long offs[4] = {r0 + c0, r0 + c1, r1 + c0, r1 + c1};
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                load_vec<16>(xg + offs[c] + rot * 16, &v[c][0]);
-                load_vec<16>(xg + offs[c] + (rot ^ 1) * 16, &v[c][4]);
-            }
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int h = 0; h < NH; ++h) load_vec<16>(xg + offs[c] + hb[h], &v[c][4 * h]);
         }
     };
 
@@ -316,6 +381,34 @@ __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc
         }
         load_fallback(t0);
     }
+#if DCN_BAND_AHEAD == 2
+    // geometry two taps ahead of the math: tap k + 2's chain of dependent
+    // instructions runs while tap k is accumulated and tap k + 1 loads
+    Tap tn;
+    if (K > 1) tn = geometry();
+#pragma unroll UNROLL
+    for (int k = 0; k < K; ++k) {
+        const bool more = k + 1 < K;
+        Tap tnn;
+        if (k + 2 < K) tnn = geometry();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                float f[8];
+                widen<T, 8>(&v[c][4 * h], f);
+                axpy<8>(acc + 8 * h, w[c], f);
+            }
+            if (more) load_shared(tn, c);
+        }
+        if (more) {
+            load_fallback(tn);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) w[c] = tn.w[c];
+        }
+        tn = tnn;
+    }
+#else
 #pragma unroll UNROLL
     for (int k = 0; k < K; ++k) {
         const bool more = k + 1 < K;
@@ -323,11 +416,12 @@ __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc
         if (more) tn = geometry();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            float f[8];
-            widen<T, 8>(&v[c][0], f);
-            axpy<8>(acc, w[c], f);
-            widen<T, 8>(&v[c][4], f);
-            axpy<8>(acc + 8, w[c], f);
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                float f[8];
+                widen<T, 8>(&v[c][4 * h], f);
+                axpy<8>(acc + 8 * h, w[c], f);
+            }
             if (more) load_shared(tn, c);
         }
         if (more) {
@@ -336,16 +430,16 @@ __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc
             for (int c = 0; c < 4; ++c) w[c] = tn.w[c];
         }
     }
+#endif
 
-    // acc[0..7] holds the half at byte rot * 16 of the group, acc[8..15] the other
-    uint32_t o0[4], o1[4];
-    narrow<T, 8>(acc, o0);
-    narrow<T, 8>(acc + 8, o1);
+    // acc[8h .. 8h + 7] holds the half at byte hb[h] of the group
     char* ob = static_cast<char*>(a.out) +
                (((long long)n * a.Ho + oy) * row_items + item) * 32;
-    if (active) {
-        store_vec<16>(ob + rot * 16, o0);
-        store_vec<16>(ob + (rot ^ 1) * 16, o1);
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+        uint32_t o[4];
+        narrow<T, 8>(acc + 8 * h, o);
+        if (active) store_vec<16>(ob + hb[h], o);
     }
 }
 
@@ -353,19 +447,22 @@ __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc
 
 template <typename T, bool SOFTMAX, int KF>
 __global__ void __launch_bounds__(kBandMaxThreads, 1) dcn_band_kernel(const BandArgs a) {
+    constexpr int LPI = kBandLanesPerItem;
+    constexpr int RUN = 32 / LPI;          // items per warp run
     static_assert(sizeof(T) == 2, "the band kernel handles 16-bit data");
     extern __shared__ __align__(128) unsigned char band_smem[];
+    const int NS = a.stages;
     unsigned char* ring = band_smem;
     unsigned char* stages = band_smem + a.ring_bytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(stages + kBandStages * a.stage_bytes);
-    uint64_t* empty = full + kBandStages;
-    int* descs = reinterpret_cast<int*>(empty + kBandStages);
+    uint64_t* full = reinterpret_cast<uint64_t*>(stages + NS * a.stage_bytes);
+    uint64_t* empty = full + NS;
+    int* descs = reinterpret_cast<int*>(empty + NS);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nc = a.consumer_warps;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kBandStages; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], (uint32_t)nc);
         }
@@ -402,22 +499,22 @@ __global__ void __launch_bounds__(kBandMaxThreads, 1) dcn_band_kernel(const Band
             }
             const int v_hi = v_lo + (y_hi - y_lo);
             const int v_first_new = v_lo + (first_new - y_lo);
-            // free the stage buffer (step - kBandStages) and every ring slot
+            // free the stage buffer (step - NS) and every ring slot
             // that the new rows overwrite (steps whose band starts at or below
             // v_hi - RB)
             while (done < step - 1) {
                 const int t = done + 1;
                 const BandDesc* dt =
-                    reinterpret_cast<const BandDesc*>(descs + (t % kBandStages) * kBandDescInts);
-                const bool must = t <= step - kBandStages ||
+                    reinterpret_cast<const BandDesc*>(descs + (t % NS) * kBandDescInts);
+                const bool must = t <= step - NS ||
                                   (first_new <= y_hi && dt->v_lo <= v_hi - RB);
                 if (!must) break;
-                if (!mbar_wait(&empty[t % kBandStages], (uint32_t)((t / kBandStages) & 1),
+                if (!mbar_wait(&empty[t % NS], (uint32_t)((t / NS) & 1),
                                a.error))
                     return;
                 done = t;
             }
-            const int sb = step % kBandStages;
+            const int sb = step % NS;
             BandDesc* d = reinterpret_cast<BandDesc*>(descs + sb * kBandDescInts);
             d->y_lo = y_lo;
             d->y_hi = y_hi;
@@ -454,8 +551,8 @@ __global__ void __launch_bounds__(kBandMaxThreads, 1) dcn_band_kernel(const Band
             cur += st.nrows;
         }
         // leave only once the copies of the last stages have landed
-        for (int t = max(0, step - kBandStages); t < step; ++t)
-            if (!mbar_wait(&full[t % kBandStages], (uint32_t)((t / kBandStages) & 1), a.error))
+        for (int t = max(0, step - NS); t < step; ++t)
+            if (!mbar_wait(&full[t % NS], (uint32_t)((t / NS) & 1), a.error))
                 return;
         return;
     }
@@ -473,10 +570,10 @@ __global__ void __launch_bounds__(kBandMaxThreads, 1) dcn_band_kernel(const Band
     for (int cur = r_begin; cur < r_end; ++step) {
         const BandStep st = band_step(a, cur, r_end);
         cur += st.nrows;
-        const int sb = step % kBandStages;
-        if (!mbar_wait(&full[sb], (uint32_t)((step / kBandStages) & 1), a.error)) return;
+        const int sb = step % NS;
+        if (!mbar_wait(&full[sb], (uint32_t)((step / NS) & 1), a.error)) return;
         const BandDesc dsc = *reinterpret_cast<const BandDesc*>(descs + sb * kBandDescInts);
-        const unsigned char* sbuf = stages + sb * a.stage_bytes;
+        const uint32_t sbuf_s = smem_u32(stages + sb * a.stage_bytes);
         const int runs = st.nrows * a.runs_per_row;
         const int r_first = (warp - j0 % nc + nc) % nc;
         j0 += runs;
@@ -485,16 +582,16 @@ __global__ void __launch_bounds__(kBandMaxThreads, 1) dcn_band_kernel(const Band
             const int run_in_row = r - row_local * a.runs_per_row;
             // lanes past the end of the row compute a copy of the row's last
             // item and store nothing (every lane takes part in the warp votes)
-            const bool active = run_in_row * 32 + lane < row_items;
-            const int item = active ? run_in_row * 32 + lane : row_items - 1;
+            const bool active = run_in_row * RUN + lane / LPI < row_items;
+            const int item = active ? run_in_row * RUN + lane / LPI : row_items - 1;
             const int oy = st.o + row_local;
-            const T* offp = reinterpret_cast<const T*>(sbuf + row_local * a.off_row_bytes) +
-                            (long long)item * K * 2;
-            const T* maskp = reinterpret_cast<const T*>(sbuf + a.th * a.off_row_bytes +
-                                                        row_local * a.mask_row_bytes) +
-                             (long long)item * K;
-            band_item<T, T, SOFTMAX, KF>(a, dsc, ring_s, st.n, oy, item, active, offp, maskp,
-                                         lane);
+            const uint32_t off_s = sbuf_s + row_local * a.off_row_bytes +
+                                   (uint32_t)(item * K * 2 * (int)sizeof(T));
+            const uint32_t mask_s = sbuf_s + a.th * a.off_row_bytes +
+                                    row_local * a.mask_row_bytes +
+                                    (uint32_t)(item * K * (int)sizeof(T));
+            band_item<T, T, SOFTMAX, KF, LPI>(a, dsc, ring_s, st.n, oy, item, active, off_s,
+                                              mask_s, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[sb]);

@@ -36,8 +36,7 @@
 namespace dcnb {
 
 constexpr int kFusedEpilogueWarps = 4;
-constexpr int kFusedMaxThreads = 32 * 16;
-constexpr int kFusedStages = 2;        // A tiles, TMEM accumulators, om buffers
+constexpr int kFusedMaxThreads = 32 * 16;   // samplers, producer, MMA, 4 epilogue warps
 
 struct BandFusedArgs {
     CUtensorMap tmap_x;        // x viewed as [N*H*W rows][C], box {64, a_rows}, 128-byte swizzle
@@ -50,7 +49,7 @@ struct BandFusedArgs {
     int a_rows;                // th * W: pixels (rows) of one A tile load
     int consumer_warps;        // sampler warps
     uint32_t tmem_cols;        // TMEM columns allocated (power of 2 >= 2 * NJ)
-    uint32_t a_bytes;          // one A stage: kchunks * 128 rows * 128 B
+    uint32_t a_bytes;          // one A stage: kchunks * 128-byte K slices of a_stage_rows rows
     uint32_t a_box_bytes;      // bytes one step's A loads deliver: kchunks * a_rows * 128
     uint32_t w_bytes;          // kchunks * NJ * 128 B
     uint32_t om_stride;        // floats per pixel in the om buffer (J rounded up to 4)
@@ -129,26 +128,29 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 template <typename T, int KF>
 __global__ void __launch_bounds__(kFusedMaxThreads, 1)
     dcn_band_fused_kernel(const __grid_constant__ BandFusedArgs f) {
+    constexpr int LPI = kBandLanesPerItem;
+    constexpr int RUN = 32 / LPI;          // items per warp run
     const BandArgs& a = f.b;
+    const int NS = a.stages;               // steps in flight: A tiles, accumulators, om buffers
     extern __shared__ __align__(128) unsigned char fused_smem[];
     // 1024-byte aligned base for the swizzled tiles (the allocation has 1 KB of slack)
     const uint32_t raw = smem_u32(fused_smem);
     unsigned char* base = fused_smem + ((1024u - (raw & 1023u)) & 1023u);
     unsigned char* wtile = base;                                     // w_bytes
-    unsigned char* atile = wtile + f.w_bytes;                        // 2 x a_bytes
-    unsigned char* ring = atile + kFusedStages * f.a_bytes;          // ring_bytes
-    float* om = reinterpret_cast<float*>(ring + a.ring_bytes);       // 2 x om_bytes
+    unsigned char* atile = wtile + f.w_bytes;                        // NS x a_bytes
+    unsigned char* ring = atile + NS * f.a_bytes;          // ring_bytes
+    float* om = reinterpret_cast<float*>(ring + a.ring_bytes);       // NS x om_bytes
     uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(om) +
-                                                 kFusedStages * f.om_bytes);
+                                                 NS * f.om_bytes);
     uint64_t* full = bars;                          // ring rows + A tile of a step
-    uint64_t* empty = full + kBandStages;           // samplers done with a step
-    uint64_t* mma_done = empty + kBandStages;       // accumulator stage written
-    uint64_t* tmem_free = mma_done + kFusedStages;  // accumulator stage read
-    uint64_t* om_full = tmem_free + kFusedStages;   // om buffer written
-    uint64_t* om_free = om_full + kFusedStages;     // om buffer read
-    uint64_t* w_full = om_free + kFusedStages;      // weight tile landed
+    uint64_t* empty = full + NS;           // samplers done with a step
+    uint64_t* mma_done = empty + NS;       // accumulator stage written
+    uint64_t* tmem_free = mma_done + NS;  // accumulator stage read
+    uint64_t* om_full = tmem_free + NS;   // om buffer written
+    uint64_t* om_free = om_full + NS;     // om buffer read
+    uint64_t* w_full = om_free + NS;      // weight tile landed
     int* descs = reinterpret_cast<int*>(w_full + 1);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(descs + kBandStages * kBandDescInts);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(descs + NS * kBandDescInts);
     float* bias_s = reinterpret_cast<float*>(tmem_slot + 4);       // NJ floats
 
     const int warp = threadIdx.x >> 5;
@@ -157,11 +159,11 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
     const int w_prod = nc, w_mma = nc + 1, w_epi = nc + 2;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kBandStages; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], (uint32_t)nc);
         }
-        for (int s = 0; s < kFusedStages; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&mma_done[s], 1);
             mbar_init(&tmem_free[s], kFusedEpilogueWarps);
             mbar_init(&om_full[s], kFusedEpilogueWarps);
@@ -216,11 +218,11 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
                 while (done < step - 1) {
                     const int t = done + 1;
                     const BandDesc* dt = reinterpret_cast<const BandDesc*>(
-                        descs + (t % kBandStages) * kBandDescInts);
-                    const bool must = t <= step - kBandStages ||
+                        descs + (t % NS) * kBandDescInts);
+                    const bool must = t <= step - NS ||
                                       (first_new <= y_hi && dt->v_lo <= v_hi - RB);
                     if (!must) break;
-                    if (!mbar_wait(&empty[t % kBandStages], (uint32_t)((t / kBandStages) & 1),
+                    if (!mbar_wait(&empty[t % NS], (uint32_t)((t / NS) & 1),
                                    a.error)) {
                         ok = false;
                         break;
@@ -228,7 +230,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
                     done = t;
                 }
                 if (!ok) break;
-                const int sb = step % kBandStages;
+                const int sb = step % NS;
                 BandDesc* d = reinterpret_cast<BandDesc*>(descs + sb * kBandDescInts);
                 d->y_lo = y_lo;
                 d->y_hi = y_hi;
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
                 }
                 // the step's pixels: rows (n H + o) W ... of the 2-D view of x
                 const int prow = (st.n * a.H + st.o) * a.W;
-                unsigned char* adst = atile + (step % kFusedStages) * f.a_bytes;
+                unsigned char* adst = atile + (step % NS) * f.a_bytes;
                 for (int kc = 0; kc < f.kchunks; ++kc)
                     tma_load_2d(adst + kc * (f.a_bytes / f.kchunks), &f.tmap_x, kc * 64, prow,
                                 &full[sb]);
@@ -263,8 +265,8 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
                 cur += st.nrows;
             }
             // leave the loop only once the last stages' copies have landed
-            for (int t = max(0, step - kBandStages); t < step; ++t)
-                (void)mbar_wait(&full[t % kBandStages], (uint32_t)((t / kBandStages) & 1),
+            for (int t = max(0, step - NS); t < step; ++t)
+                (void)mbar_wait(&full[t % NS], (uint32_t)((t / NS) & 1),
                                 a.error);
             (void)mbar_wait(w_full, 0, a.error);
         }
@@ -278,10 +280,10 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
             for (int cur = r_begin; cur < r_end && ok; ++step) {
                 const BandStep st = band_step(a, cur, r_end);
                 cur += st.nrows;
-                const int sb = step % kBandStages, fs = step % kFusedStages;
-                if (!mbar_wait(&full[sb], (uint32_t)((step / kBandStages) & 1), a.error)) break;
-                if (step >= kFusedStages &&
-                    !mbar_wait(&tmem_free[fs], (uint32_t)(((step / kFusedStages) - 1) & 1),
+                const int sb = step % NS, fs = step % NS;
+                if (!mbar_wait(&full[sb], (uint32_t)((step / NS) & 1), a.error)) break;
+                if (step >= NS &&
+                    !mbar_wait(&tmem_free[fs], (uint32_t)(((step / NS) - 1) & 1),
                                a.error))
                     break;
                 tmem_fence_after();
@@ -308,10 +310,10 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
         for (int cur = r_begin; cur < r_end; ++step) {
             const BandStep st = band_step(a, cur, r_end);
             cur += st.nrows;
-            const int fs = step % kFusedStages;
-            if (!mbar_wait(&mma_done[fs], (uint32_t)((step / kFusedStages) & 1), a.error)) break;
-            if (step >= kFusedStages &&
-                !mbar_wait(&om_free[fs], (uint32_t)(((step / kFusedStages) - 1) & 1), a.error))
+            const int fs = step % NS;
+            if (!mbar_wait(&mma_done[fs], (uint32_t)((step / NS) & 1), a.error)) break;
+            if (step >= NS &&
+                !mbar_wait(&om_free[fs], (uint32_t)(((step / NS) - 1) & 1), a.error))
                 break;
             tmem_fence_after();
             float* dst = om + (size_t)fs * (f.om_bytes / 4) + (size_t)pix * f.om_stride;
@@ -352,25 +354,26 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
         for (int cur = r_begin; cur < r_end; ++step) {
             const BandStep st = band_step(a, cur, r_end);
             cur += st.nrows;
-            const int sb = step % kBandStages, fs = step % kFusedStages;
-            if (!mbar_wait(&full[sb], (uint32_t)((step / kBandStages) & 1), a.error)) break;
-            if (!mbar_wait(&om_full[fs], (uint32_t)((step / kFusedStages) & 1), a.error)) break;
+            const int sb = step % NS, fs = step % NS;
+            if (!mbar_wait(&full[sb], (uint32_t)((step / NS) & 1), a.error)) break;
+            if (!mbar_wait(&om_full[fs], (uint32_t)((step / NS) & 1), a.error)) break;
             const BandDesc dsc = *reinterpret_cast<const BandDesc*>(descs + sb * kBandDescInts);
-            const float* omb = om + (size_t)fs * (f.om_bytes / 4);
+            const uint32_t omb_s = smem_u32(om) + (uint32_t)fs * f.om_bytes;
             const int runs = st.nrows * a.runs_per_row;
             const int r_first = (warp - j0 % nc + nc) % nc;
             j0 += runs;
             for (int r = r_first; r < runs; r += nc) {
                 const int row_local = (int)a.div_runs.div((uint32_t)r);
                 const int run_in_row = r - row_local * a.runs_per_row;
-                const bool active = run_in_row * 32 + lane < row_items;
-                const int item = active ? run_in_row * 32 + lane : row_items - 1;
+                const bool active = run_in_row * RUN + lane / LPI < row_items;
+                const int item = active ? run_in_row * RUN + lane / LPI : row_items - 1;
                 const int ox = (int)a.div_G.div((uint32_t)item);
                 const int g = item - ox * a.G;
-                const float* prow = omb + (size_t)(row_local * a.W + ox) * f.om_stride;
-                band_item<T, float, false, KF>(a, dsc, ring_s, st.n, st.o + row_local, item,
-                                               active, prow + g * 2 * K, prow + 2 * GK + g * K,
-                                               lane);
+                const uint32_t prow =
+                    omb_s + (uint32_t)((row_local * a.W + ox) * f.om_stride) * 4u;
+                band_item<T, float, false, KF, LPI>(a, dsc, ring_s, st.n, st.o + row_local,
+                                                    item, active, prow + (uint32_t)(g * 2 * K) * 4u,
+                                                    prow + (uint32_t)(2 * GK + g * K) * 4u, lane);
             }
             __syncwarp();
             if (lane == 0) {

@@ -58,7 +58,8 @@ def test_dcn_backward_workload_full_size(name):
     w = gen.WORKLOADS[name]
     inp = dcn_problem(w, seed=0)
     got = run_dcn_bwd(inp, w)
-    for n in sorted({0, w.N - 1}):
+    # first, middle (where the persistent CTAs' ranges meet) and last image
+    for n in sorted({0, w.N // 2, w.N - 1}):
         check_dcn(got, ref_dcn_bwd(inp, w, n), f"{name} image {n}", n)
 
 

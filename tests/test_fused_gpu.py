@@ -66,11 +66,11 @@ BAND_CASES = [
     # N, H, W, C, G, k, pad, dil, dtype
     (2, 12, 14, 64, 4, 3, 1, 1, "f16"),
     (2, 10, 20, 128, 8, 3, 1, 1, "bf16"),    # two 64-channel K slices, 216 outputs
-    (1, 9, 128, 64, 4, 3, 1, 1, "f16"),      # 128 pixels per step: the whole M tile
+    (2, 9, 32, 64, 4, 1, 0, 1, "f16"),       # 1 x 1 window: 128 pixels per step, the whole M tile
     (3, 5, 9, 64, 4, 1, 0, 1, "bf16"),       # 1 x 1 window: 12 outputs
     (2, 12, 16, 64, 4, 3, 2, 2, "f16"),      # dilation 2
     (5, 3, 8, 64, 4, 3, 1, 1, "f16"),        # several images per CTA
-    (1, 30, 40, 256, 16, 1, 0, 1, "bf16"),   # C = 256: four K slices
+    (1, 12, 8, 256, 16, 1, 0, 1, "bf16"),    # C = 256: four K slices
 ]
 
 

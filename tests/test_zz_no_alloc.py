@@ -1,5 +1,6 @@
 """dcn_backward_static_scratch: the backward with the library's own static
-grad_x accumulator, against dcn_backward with a caller workspace.
+grad_x accumulator, against dcn_backward with a caller workspace and against
+the float64 oracle's gradients.
 
 Collected last on purpose: it must pass both in a fresh process (where its
 first call looks up the accumulator's device address) and after every other
@@ -14,6 +15,7 @@ import torch
 import deformable_attention_sampling_b200 as dcnb
 from deformable_attention_sampling_b200 import build as dcn_build
 import gen
+import oracle
 from tests.parity import compare
 
 DEV = "cuda:0"
@@ -43,6 +45,8 @@ def test_static_scratch_matches_the_workspace_entry(dt, sm):
     host["grad_out"] = gen.grad_out((w.N, w.Ho, w.Wo, w.C), w.dtype, seed=21)
     t = {k: v.to(DEV) for k, v in host.items()}
 
+    exact = oracle.dcn_backward_ref(host["x"], host["offset"], host["mask"], host["grad_out"],
+                                    w.kh, w.kw, w.stride, w.pad, w.dil, w.softmax_flag)
     ref = _empty_grads(t)
     code = gen.DTYPE_CODES[dt]
     nbytes = dcnb.dcn_backward_workspace_size(w.N, w.H, w.W, w.C, code)
@@ -57,8 +61,9 @@ def test_static_scratch_matches_the_workspace_entry(dt, sm):
         dcnb.dcn_backward_static_scratch(*_args(w, t, got))
         torch.cuda.synchronize()
         assert dcnb.dcn_launch_count() - before == (3 if dt != "f32" else 2)
-        for name, g, r in zip(("grad_x", "grad_offset", "grad_mask"), got, ref):
+        for name, g, r, e in zip(("grad_x", "grad_offset", "grad_mask"), got, ref, exact):
             compare(g, r.double().cpu().numpy(), f"{dt} call {call} {name}")
+            compare(g, e, f"{dt} call {call} {name} vs the oracle")
         # the per-tap gradients are deterministic: bit for bit the same
         assert torch.equal(got[1], ref[1]) and torch.equal(got[2], ref[2])
 
