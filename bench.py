@@ -51,8 +51,8 @@ SMEM_BYTES_PER_CLK = 128.0
 # dram__bytes_write.sum per launch, headline workload), with the hash of the
 # files the headline launch is built from; reported as null once they change.
 NCU_TRAFFIC = {
-    "source_sha256": "4759a5db507e1eb4cf2c92f0e46ac3da631aa04d770c1be48ca6718f61af10c5",
-    "bytes_per_launch": 69190144 + 3826688,   # DRAM read + write, one headline launch
+    "source_sha256": "903eb45612d69b1b54e3254a75f26395c21cfcaf45eb8dc857a067e95c12028a",
+    "bytes_per_launch": 69523456 + 4337408,   # DRAM read + write, one headline launch
 }
 
 # What the headline dcn_forward launch is built from: its device code and the
@@ -473,7 +473,7 @@ class MsdaPointsRunner:
 class FusedRunner:
     """One step = one dcnv4_fused_forward call (merged offset / mask linear on
     the tensor cores feeding the sampler; offsets never leave the SM)."""
-    kernel = "dcn_fwd_kernel (fused front end)"
+    kernel = "dcn_band_fused_kernel (tcgen05 front end) where it applies, else dcn_fwd_kernel"
 
     def __init__(self, w, seed, device):
         import deformable_attention_sampling_b200 as dcnb
@@ -701,6 +701,17 @@ def run_b200(args):
             torch.cuda.synchronize(device)
             del probe
         runner.kernel = "dcn_band_kernel" if band else "dcn_fwd_kernel"
+    elif isinstance(runner, FusedRunner):
+        probe = runner.alloc_set()
+        fused_band = dcnb.library().dcnv4_fused_forward_algo(
+            probe["x"].data_ptr(), probe["w_om"].data_ptr(), probe["b_om"].data_ptr(),
+            probe["out"].data_ptr(), w.N, w.H, w.W, w.C, w.G, w.kh, w.kw, w.pad, w.dil,
+            runner.code, dcnb.DCN_ALGO_BAND,
+            int(torch.cuda.current_stream(device).cuda_stream)) == 0
+        torch.cuda.synchronize(device)
+        del probe
+        runner.kernel = ("dcn_band_fused_kernel (tcgen05 front end)" if fused_band
+                         else "dcn_fwd_kernel (fused front end, mma.sync)")
     bytes_per_step = runner.bytes_per_step()
     l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
     n_sets = max(2, int(np.ceil(3 * l2_bytes / bytes_per_step)))
