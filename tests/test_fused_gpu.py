@@ -83,7 +83,8 @@ def test_fused_band_kernel_small_shapes(case):
     expect = ref(inp, w)
     band = run(inp, w, algo="band")
     compare(band, expect, f"{case} band")
-    compare(run(inp, w, algo="gather"), expect, f"{case} gather")
+    if C <= 128:   # the gather kernel's per-warp linear holds at most 128 channels
+        compare(run(inp, w, algo="gather"), expect, f"{case} gather")
     assert torch.equal(run(inp, w, algo="auto"), band)
 
 
