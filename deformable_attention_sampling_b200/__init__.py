@@ -33,7 +33,13 @@ from ._binding import (  # noqa: F401
     dcn_backward_workspace_size,
     dcn_forward,
     dcn_forward_algo,
-    dcn_forward_timeouts,
+    DCN_FLAG_BAD_LEVELS,
+    DCN_FLAG_OUT_OF_BOUNDS,
+    DCN_FLAG_WAIT_TIMEOUT,
+    DEBUG_LIB_PATH,
+    dcn_debug_checks,
+    dcn_device_flags,
+    debug_library,
     dcn_grad,
     dcn_last_cuda_error,
     dcn_launch_count,

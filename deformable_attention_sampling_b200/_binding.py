@@ -14,6 +14,7 @@ import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "_lib", "libdcn_b200.so")
+DEBUG_LIB_PATH = os.path.join(PKG, "_lib", "libdcn_b200_debug.so")
 
 DCN_OK = 0
 DCN_ERR_INVALID_ARG = -1
@@ -21,6 +22,14 @@ DCN_ERR_UNSUPPORTED = -2
 DCN_ERR_MISALIGNED = -3
 DCN_ERR_CUDA = -4
 DTYPE_CODES = {"f32": 0, "f16": 1, "bf16": 2}
+DCN_FLAG_WAIT_TIMEOUT = 1
+DCN_FLAG_OUT_OF_BOUNDS = 2
+DCN_FLAG_BAD_LEVELS = 4
+# the entry points the debug library holds (the forward calls and the status calls)
+DEBUG_SYMBOLS = ("dcn_forward", "dcn_forward_algo", "dcnv4_fused_forward",
+                 "dcnv4_fused_forward_algo", "msda_forward", "msda_forward_points",
+                 "msda_mask_value", "dcn_output_size", "dcn_status_string", "dcn_last_cuda_error",
+                 "dcn_launch_count", "dcn_device_flags", "dcn_debug_checks", "dcn_version")
 DCN_ALGO_AUTO = 0
 DCN_ALGO_GATHER = 1
 DCN_ALGO_BAND = 2
@@ -33,7 +42,8 @@ _LL = ctypes.c_longlong
 SIGNATURES = {
     "dcn_forward": (_I, [_VP, _VP, _VP, _VP] + [_I] * 12 + [_VP]),
     "dcn_forward_algo": (_I, [_VP, _VP, _VP, _VP] + [_I] * 13 + [_VP]),
-    "dcn_forward_timeouts": (_I, []),
+    "dcn_device_flags": (_I, [_I]),
+    "dcn_debug_checks": (_I, []),
     "msda_forward": (_I, [_VP] * 6 + [_I] * 7 + [_VP]),
     "msda_forward_points": (_I, [_VP] * 4 + [_I] + [_VP] * 4 + [_I] * 7 + [_VP]),
     "msda_mask_value": (_I, [_VP] * 3 + [_I] * 5 + [_VP]),
@@ -88,6 +98,28 @@ def library():
     return _load()
 
 
+_debug_lib = None
+
+
+def debug_library():
+    """The debug library (libdcn_b200_debug.so: the forward and status calls
+    with device-side address and level-table checks), loaded on first use."""
+    global _debug_lib
+    if _debug_lib is None:
+        if not os.path.exists(DEBUG_LIB_PATH):
+            raise RuntimeError(
+                f"{DEBUG_LIB_PATH} is missing: build it with "
+                "`python -m deformable_attention_sampling_b200.build`")
+        lib = ctypes.CDLL(DEBUG_LIB_PATH)
+        for name in DEBUG_SYMBOLS:
+            res, args = SIGNATURES[name]
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _debug_lib = lib
+    return _debug_lib
+
+
 def _ptr(p):
     if p is None:
         return None
@@ -128,13 +160,19 @@ def dcn_forward_algo(x, offset, mask, out, N, H, W, C, G, kh, kw, stride, pad, d
            "dcn_forward_algo")
 
 
-def dcn_forward_timeouts():
-    """C dcn_forward_timeouts: the band kernel's timed-out-wait word on the
-    current device (0 when no wait ever ran out); synchronous."""
-    r = _load().dcn_forward_timeouts()
+def dcn_device_flags(reset=False, lib=None):
+    """C dcn_device_flags: the status word of the current device (DCN_FLAG_*
+    bits), cleared when reset; synchronous.  `lib`: the debug library handle
+    instead of the release library."""
+    r = (lib or _load()).dcn_device_flags(1 if reset else 0)
     if r < 0:
-        raise DcnError(r, "dcn_forward_timeouts")
+        raise DcnError(r, "dcn_device_flags")
     return r
+
+
+def dcn_debug_checks(lib=None):
+    """1 for the debug library (device-side checks), 0 for the release one."""
+    return int((lib or _load()).dcn_debug_checks())
 
 
 def msda_forward(value, spatial_shapes, level_start, sampling_loc, attn_w, out, N, Lq, M, D,

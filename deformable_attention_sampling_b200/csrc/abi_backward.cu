@@ -249,6 +249,9 @@ int dcn_backward(const void* x, const void* offset, const void* mask, const void
     a.w_om = nullptr;
     a.b_om = nullptr;
     a.J = 0;
+    a.flags = device_flags_word();
+    a.x_bytes = img_bytes * N;
+    a.out_bytes = out_img_bytes * N;
     b.grad_out = grad_out;
     b.grad_offset = grad_offset;
     b.grad_mask = grad_mask;
@@ -362,6 +365,7 @@ int msda_backward(const void* value, const int64_t* spatial_shapes, const int64_
     a.div_tpi = make_div((uint32_t)tpi);
     a.ref = nullptr;
     a.vr = nullptr;
+    a.flags = device_flags_word();
     b.grad_out = grad_out;
     b.grad_loc = grad_loc;
     b.grad_attn = grad_attn;

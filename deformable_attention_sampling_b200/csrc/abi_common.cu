@@ -113,15 +113,15 @@ int wave_size(const void* fn, int threads, int smem) {
 // L1 reuse dominates and tiles grow up to kDcnMaxWarps rows (one CTA per SM).
 constexpr int kSmallMapRows = 64;
 
-// Timeout word of the band kernel's bounded waits, one per device; its
-// device address is looked up once per device.
-__device__ unsigned int g_band_timeouts;
+// Status word of the kernels (DCN_FLAG_* bits), one per device; its device
+// address is looked up once per device.
+__device__ unsigned int g_device_flags;
 
 constexpr int kMaxScratchDevices = 64;
 std::mutex g_timeout_mutex;
 unsigned int* g_timeout_ptr[kMaxScratchDevices] = {};
 
-unsigned int* band_timeout_word() {
+unsigned int* device_flags_word() {
     int device = 0;
     if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxScratchDevices) {
         (void)cudaGetLastError();
@@ -130,7 +130,7 @@ unsigned int* band_timeout_word() {
     std::lock_guard<std::mutex> lock(g_timeout_mutex);
     if (g_timeout_ptr[device] == nullptr) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_band_timeouts) != cudaSuccess) {
+        if (cudaGetSymbolAddress(&p, g_device_flags) != cudaSuccess) {
             (void)cudaGetLastError();
             return nullptr;
         }
@@ -215,13 +215,28 @@ const char* dcn_status_string(int status) {
     }
 }
 
-int dcn_forward_timeouts(void) {
+int dcn_device_flags(int reset) {
     unsigned int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_band_timeouts, sizeof(v)) != cudaSuccess) {
+    if (cudaMemcpyFromSymbol(&v, g_device_flags, sizeof(v)) != cudaSuccess) {
         g_last_cuda_error = (int)cudaGetLastError();
         return DCN_ERR_CUDA;
     }
+    if (reset) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_flags, &zero, sizeof(zero)) != cudaSuccess) {
+            g_last_cuda_error = (int)cudaGetLastError();
+            return DCN_ERR_CUDA;
+        }
+    }
     return (int)(v & 0x7fffffffu);
+}
+
+int dcn_debug_checks(void) {
+#ifdef DCN_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 int dcn_last_cuda_error(void) { return g_last_cuda_error; }

@@ -133,9 +133,9 @@ TileShape choose_tile(int N, int Ho, int runs, int kernel_extent, int sms, int c
 // elements read as zero.  The encoder comes from the driver through the
 // runtime's entry-point query (no link-time dependency on libcuda).  False on
 // any error.
-// Device address of the timeout word of the band kernels' bounded waits on
-// the current device (looked up once per device), or null.
-unsigned int* band_timeout_word();
+// Device address of the kernels' status word (DCN_FLAG_* bits) on the current
+// device (looked up once per device), or null.
+unsigned int* device_flags_word();
 
 bool encode_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner,
                     uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);

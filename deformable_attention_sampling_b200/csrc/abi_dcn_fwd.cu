@@ -101,7 +101,9 @@ bool band_config(const void* x, const void* offset, const void* mask, void* out,
         a->div_G = make_div((uint32_t)G);
         a->div_Ho = make_div((uint32_t)Ho);
         a->div_runs = make_div((uint32_t)runs_per_row);
-        a->error = band_timeout_word();
+        a->flags = device_flags_word();
+        a->x_bytes = (long long)N * H * row_bytes;
+        a->out_bytes = (long long)N * Ho * Wo * C * es;
         *smem = (int)bytes;
         *threads = 32 * (warps + 1);
         return true;
@@ -257,6 +259,9 @@ int dcn_forward_algo(const void* x, const void* offset, const void* mask, void* 
     a.w_om = nullptr;
     a.b_om = nullptr;
     a.J = 0;
+    a.flags = device_flags_word();
+    a.x_bytes = img_bytes * N;
+    a.out_bytes = out_img_bytes * N;
 
     const void* fn = nullptr;
     switch (dtype) {

@@ -111,7 +111,9 @@ bool band_fused_config(const void* x, const void* w_om, const void* b_om, void* 
             a.div_G = make_div((uint32_t)G);
             a.div_Ho = make_div((uint32_t)H);
             a.div_runs = make_div((uint32_t)runs_per_row);
-            a.error = nullptr;
+            a.flags = nullptr;
+            a.x_bytes = (long long)N * H * row_bytes;
+            a.out_bytes = (long long)N * H * row_bytes;
             f->b_om = b_om;
             f->J = J;
             f->NJ = NJ;
@@ -199,7 +201,7 @@ int dcnv4_fused_forward_algo(const void* x, const void* w_om, const void* b_om, 
         int smem = 0, threads = 0;
         if (band_fused_config(x, w_om, b_om, out, N, H, W, C, G, kh, kw, pad, dil,
                               dtype == DCN_BF16, &f, &smem, &threads)) {
-            f.b.error = band_timeout_word();
+            f.b.flags = device_flags_word();
             const void* fn = dtype == DCN_F16 ? band_fused_kernel_for<__half>(kh, kw)
                                               : band_fused_kernel_for<__nv_bfloat16>(kh, kw);
             // one CTA per SM (the shared-memory footprint allows no more)
@@ -279,6 +281,9 @@ int dcnv4_fused_forward_algo(const void* x, const void* w_om, const void* b_om, 
     a.w_om = w_om;
     a.b_om = b_om;
     a.J = J;
+    a.flags = device_flags_word();
+    a.x_bytes = img_bytes * N;
+    a.out_bytes = img_bytes * N;
 
     const void* fn = nullptr;
     switch (dtype) {

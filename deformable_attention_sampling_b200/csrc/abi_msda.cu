@@ -108,6 +108,7 @@ static int msda_launch(const void* value, const int64_t* spatial_shapes,
     a.div_tpi = make_div((uint32_t)tpi);
     a.ref = ref;
     a.vr = vr;
+    a.flags = device_flags_word();
 
     const void* fn = nullptr;
     switch (dtype) {

@@ -14,6 +14,27 @@
 
 namespace dcnb {
 
+// ------------------------------------------------------------ status word --
+
+// Bits of the per-device status word (dcn_device_flags in the C interface).
+constexpr unsigned int kFlagWaitTimeout = 1u;   // a bounded pipeline wait gave up
+constexpr unsigned int kFlagOutOfBounds = 2u;   // debug library: an access outside its buffer
+constexpr unsigned int kFlagBadLevels = 4u;     // debug library: an inconsistent MSDA level table
+
+__device__ __forceinline__ void set_flag(unsigned int* word, unsigned int bit) {
+    if (word) atomicOr(word, bit);
+}
+
+// In the debug library (DCN_DEBUG), `cond` states that an access lies inside
+// its buffer; when it does not, the access is reported in the status word and
+// the caller skips it.  In the release library the check compiles away.
+#ifdef DCN_DEBUG
+#define DCN_IN_BOUNDS(cond, word) \
+    ((cond) ? true : (::dcnb::set_flag((word), ::dcnb::kFlagOutOfBounds), false))
+#else
+#define DCN_IN_BOUNDS(cond, word) (true || (cond))
+#endif
+
 // ---------------------------------------------------------------- vectors --
 
 // Load VB bytes from global memory (read-only for the kernel's lifetime) into

@@ -42,7 +42,7 @@
 // memory instead, under a warp-uniform branch.
 //
 // Every wait is bounded (about two seconds of %globaltimer); a wait that
-// runs out records a timeout in the error word and the thread leaves.
+// runs out records a timeout in the status word and the thread leaves.
 #pragma once
 
 #include <type_traits>
@@ -102,7 +102,9 @@ struct BandArgs {
     uint32_t ring_bytes;      // ring_rows * row_bytes (128-byte multiple)
     uint32_t stage_bytes;     // th * (off_row_bytes + mask_row_bytes), 128-byte multiple
     FastDiv div_G, div_Ho, div_runs;
-    unsigned int* error;      // timeout word (device), or null
+    unsigned int* flags;      // status word (device), or null
+    long long x_bytes;        // bytes of x and of out (bounds of the debug library's checks)
+    long long out_bytes;
 };
 
 __host__ __device__ inline int band_rows(int th, int stride, int kh, int dil, int margin) {
@@ -158,7 +160,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (global_ns() - t0 > kBandWaitNs) {
-            if (err) atomicOr(err, 1u);
+            set_flag(err, kFlagWaitTimeout);
             return false;
         }
     }
@@ -351,7 +353,15 @@ __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc
     uint32_t v[4][4 * NH];
     auto load_shared = [&](const Tap& t, int c) {
 #pragma unroll
-        for (int h = 0; h < NH; ++h) lds128(h ? t.s[c] + dh : t.s[c], &v[c][4 * h]);
+        for (int h = 0; h < NH; ++h) {
+            const uint32_t ad = h ? t.s[c] + dh : t.s[c];
+            if (DCN_IN_BOUNDS(ad >= ring_s && ad + 16 <= ring_s + a.ring_bytes, a.flags)) {
+                lds128(ad, &v[c][4 * h]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) v[c][4 * h + i] = 0u;
+            }
+        }
     };
     auto load_fallback = [&](const Tap& t) {
         if (__any_sync(0xffffffffu, t.fb) && t.fb) {
@@ -367,7 +377,16 @@ __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
-                for (int h = 0; h < NH; ++h) load_vec<16>(xg + offs[c] + hb[h], &v[c][4 * h]);
+                for (int h = 0; h < NH; ++h) {
+                    const char* src = xg + offs[c] + hb[h];
+                    const char* x0p = static_cast<const char*>(a.x);
+                    if (DCN_IN_BOUNDS(src >= x0p && src + 16 <= x0p + a.x_bytes, a.flags)) {
+                        load_vec<16>(src, &v[c][4 * h]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) v[c][4 * h + i] = 0u;
+                    }
+                }
         }
     };
 
@@ -439,7 +458,10 @@ __device__ __forceinline__ void band_item(const BandArgs& a, const BandDesc& dsc
     for (int h = 0; h < NH; ++h) {
         uint32_t o[4];
         narrow<T, 8>(acc + 8 * h, o);
-        if (active) store_vec<16>(ob + hb[h], o);
+        char* dst = ob + hb[h];
+        const char* o0p = static_cast<const char*>(a.out);
+        if (active && DCN_IN_BOUNDS(dst >= o0p && dst + 16 <= o0p + a.out_bytes, a.flags))
+            store_vec<16>(dst, o);
     }
 }
 
@@ -510,7 +532,7 @@ __global__ void __launch_bounds__(kBandMaxThreads, 1) dcn_band_kernel(const Band
                                   (first_new <= y_hi && dt->v_lo <= v_hi - RB);
                 if (!must) break;
                 if (!mbar_wait(&empty[t % NS], (uint32_t)((t / NS) & 1),
-                               a.error))
+                               a.flags))
                     return;
                 done = t;
             }
@@ -552,7 +574,7 @@ __global__ void __launch_bounds__(kBandMaxThreads, 1) dcn_band_kernel(const Band
         }
         // leave only once the copies of the last stages have landed
         for (int t = max(0, step - NS); t < step; ++t)
-            if (!mbar_wait(&full[t % NS], (uint32_t)((t / NS) & 1), a.error))
+            if (!mbar_wait(&full[t % NS], (uint32_t)((t / NS) & 1), a.flags))
                 return;
         return;
     }
@@ -571,7 +593,7 @@ __global__ void __launch_bounds__(kBandMaxThreads, 1) dcn_band_kernel(const Band
         const BandStep st = band_step(a, cur, r_end);
         cur += st.nrows;
         const int sb = step % NS;
-        if (!mbar_wait(&full[sb], (uint32_t)((step / NS) & 1), a.error)) return;
+        if (!mbar_wait(&full[sb], (uint32_t)((step / NS) & 1), a.flags)) return;
         const BandDesc dsc = *reinterpret_cast<const BandDesc*>(descs + sb * kBandDescInts);
         const uint32_t sbuf_s = smem_u32(stages + sb * a.stage_bytes);
         const int runs = st.nrows * a.runs_per_row;

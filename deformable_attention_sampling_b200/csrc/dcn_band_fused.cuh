@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
                                       (first_new <= y_hi && dt->v_lo <= v_hi - RB);
                     if (!must) break;
                     if (!mbar_wait(&empty[t % NS], (uint32_t)((t / NS) & 1),
-                                   a.error)) {
+                                   a.flags)) {
                         ok = false;
                         break;
                     }
@@ -267,13 +267,13 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
             // leave the loop only once the last stages' copies have landed
             for (int t = max(0, step - NS); t < step; ++t)
                 (void)mbar_wait(&full[t % NS], (uint32_t)((t / NS) & 1),
-                                a.error);
-            (void)mbar_wait(w_full, 0, a.error);
+                                a.flags);
+            (void)mbar_wait(w_full, 0, a.flags);
         }
     } else if (warp == w_mma) {
         // --------------------------------------------------------------- MMA
         if (lane == 0) {
-            bool ok = mbar_wait(w_full, 0, a.error);
+            bool ok = mbar_wait(w_full, 0, a.flags);
             const uint32_t idesc = umma_idesc_f16<T>(f.NJ);
             const uint32_t w_s = smem_u32(wtile);
             int step = 0;
@@ -281,10 +281,10 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
                 const BandStep st = band_step(a, cur, r_end);
                 cur += st.nrows;
                 const int sb = step % NS, fs = step % NS;
-                if (!mbar_wait(&full[sb], (uint32_t)((step / NS) & 1), a.error)) break;
+                if (!mbar_wait(&full[sb], (uint32_t)((step / NS) & 1), a.flags)) break;
                 if (step >= NS &&
                     !mbar_wait(&tmem_free[fs], (uint32_t)(((step / NS) - 1) & 1),
-                               a.error))
+                               a.flags))
                     break;
                 tmem_fence_after();
                 const uint32_t a_s = smem_u32(atile + fs * f.a_bytes);
@@ -311,9 +311,9 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
             const BandStep st = band_step(a, cur, r_end);
             cur += st.nrows;
             const int fs = step % NS;
-            if (!mbar_wait(&mma_done[fs], (uint32_t)((step / NS) & 1), a.error)) break;
+            if (!mbar_wait(&mma_done[fs], (uint32_t)((step / NS) & 1), a.flags)) break;
             if (step >= NS &&
-                !mbar_wait(&om_free[fs], (uint32_t)(((step / NS) - 1) & 1), a.error))
+                !mbar_wait(&om_free[fs], (uint32_t)(((step / NS) - 1) & 1), a.flags))
                 break;
             tmem_fence_after();
             float* dst = om + (size_t)fs * (f.om_bytes / 4) + (size_t)pix * f.om_stride;
@@ -355,8 +355,8 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1)
             const BandStep st = band_step(a, cur, r_end);
             cur += st.nrows;
             const int sb = step % NS, fs = step % NS;
-            if (!mbar_wait(&full[sb], (uint32_t)((step / NS) & 1), a.error)) break;
-            if (!mbar_wait(&om_full[fs], (uint32_t)((step / NS) & 1), a.error)) break;
+            if (!mbar_wait(&full[sb], (uint32_t)((step / NS) & 1), a.flags)) break;
+            if (!mbar_wait(&om_full[fs], (uint32_t)((step / NS) & 1), a.flags)) break;
             const BandDesc dsc = *reinterpret_cast<const BandDesc*>(descs + sb * kBandDescInts);
             const uint32_t omb_s = smem_u32(om) + (uint32_t)fs * f.om_bytes;
             const int runs = st.nrows * a.runs_per_row;

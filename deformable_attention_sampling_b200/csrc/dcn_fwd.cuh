@@ -75,6 +75,9 @@ struct DcnArgs {
     const void* w_om;         // [J][C], J = G * K * 3 (offsets in [G][K][2] order, then masks)
     const void* b_om;         // [J] or null
     int J;
+    unsigned int* flags;      // status word (device), or null
+    long long x_bytes;        // bytes of x and of out (bounds of the debug library's checks)
+    long long out_bytes;
 };
 
 // ---------------------------------------------- fused DCNv4 front end ----
@@ -455,11 +458,23 @@ __global__ void __launch_bounds__(kDcnMaxThreads, 1) dcn_fwd_kernel(const DcnArg
             }
             return t;
         };
+        // a corner load (clamped into the map, so always inside x; the debug
+        // library checks it and reads zeros instead when it is not)
+        const char* x_lo = static_cast<const char*>(a.x);
+        auto corner = [&](uint32_t off, uint32_t* dst) {
+            const char* src = xb + off;
+            if (DCN_IN_BOUNDS(src >= x_lo && src + VB <= x_lo + a.x_bytes, a.flags)) {
+                load_vec<VB>(src, dst);
+            } else {
+#pragma unroll
+                for (int i = 0; i < NW; ++i) dst[i] = 0u;
+            }
+        };
         {
             const TapGeom t0 = geometry();
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                load_vec<VB>(xb + t0.off[c], v[c]);
+                corner(t0.off[c], v[c]);
                 w[c] = t0.w[c];
             }
         }
@@ -473,7 +488,7 @@ __global__ void __launch_bounds__(kDcnMaxThreads, 1) dcn_fwd_kernel(const DcnArg
             for (int c = 0; c < 4; ++c) {
                 widen<T, CPT>(v[c], f);
                 axpy<CPT>(acc, w[c], f);
-                if (more) load_vec<VB>(xb + tn.off[c], v[c]);
+                if (more) corner(tn.off[c], v[c]);
             }
             if (more) {
 #pragma unroll
@@ -485,7 +500,9 @@ __global__ void __launch_bounds__(kDcnMaxThreads, 1) dcn_fwd_kernel(const DcnArg
         narrow<T, CPT>(acc, o);
         char* ob = static_cast<char*>(a.out) +
                    ((item_base + li) * a.D + chunk * CPT) * (int)sizeof(T);
-        store_vec<VB>(ob, o);
+        const char* o_lo = static_cast<const char*>(a.out);
+        if (DCN_IN_BOUNDS(ob >= o_lo && ob + VB <= o_lo + a.out_bytes, a.flags))
+            store_vec<VB>(ob, o);
     }
 }
 

@@ -53,6 +53,7 @@ struct MsdaArgs {
     FastDiv div_M, div_Lq, div_tpi;
     const void* ref;             // reference variants: [N][Lq][2 or 4] in valid-image units
     const void* vr;              // [N][L][2] valid ratios (W_valid / W, H_valid / H) or null
+    unsigned int* flags;         // status word (device), or null
 };
 
 // Integer cell and fraction of the normalised coordinate u on a level of
@@ -192,6 +193,25 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArg
     }
     if (threadIdx.x == 0)
         s_S = a.level_start[L - 1] + a.shapes[2 * (L - 1)] * a.shapes[2 * (L - 1) + 1];
+#ifdef DCN_DEBUG
+    // the debug library checks the level table on the device: positive shapes,
+    // levels in order without gaps from row 0; otherwise the call reads no
+    // value rows (and writes no output)
+    __shared__ int s_bad;
+    if (threadIdx.x == 0) {
+        int bad = 0;
+        long long expect = 0;
+        for (int l = 0; l < L; ++l) {
+            if (a.shapes[2 * l] <= 0 || a.shapes[2 * l + 1] <= 0 || a.level_start[l] != expect)
+                bad = 1;
+            expect = a.level_start[l] + a.shapes[2 * l] * a.shapes[2 * l + 1];
+        }
+        s_bad = bad;
+        if (bad) set_flag(a.flags, kFlagBadLevels);
+    }
+    __syncthreads();
+    if (s_bad) return;
+#endif
     __syncthreads();
 
     const int li = (int)a.div_tpi.div((uint32_t)lane);   // item within the run
@@ -282,11 +302,27 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArg
             if (nt == (nl + 1) * K) ++nl;
             return t;
         };
+        // a corner load (clamped into its level, so always inside value; the
+        // debug library checks it against the image's rows and reads zeros
+        // instead when it is not)
+        const long long img_bytes_v = s_S * pix_bytes;
+        const long long lane_off = (long long)h * a.D * (int)sizeof(T) +
+                                   (long long)chunk * CPT * (int)sizeof(T);
+        auto corner = [&](long long off, uint32_t* dst) {
+            if (DCN_IN_BOUNDS(off >= 0 && off + lane_off + VB <= img_bytes_v, a.flags)) {
+                load_vec<VB>(vb + off, dst);
+            } else {
+#pragma unroll
+                for (int i = 0; i < NW; ++i) dst[i] = 0u;
+            }
+        };
+        (void)img_bytes_v;
+        (void)lane_off;
         {
             const MsdaTap t0 = geometry();
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                load_vec<VB>(vb + t0.off[c], v[c]);
+                corner(t0.off[c], v[c]);
                 w[c] = t0.w[c];
             }
         }
@@ -300,7 +336,7 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArg
             for (int c = 0; c < 4; ++c) {
                 widen<T, CPT>(v[c], f);
                 axpy<CPT>(acc, w[c], f);
-                if (more) load_vec<VB>(vb + tn.off[c], v[c]);
+                if (more) corner(tn.off[c], v[c]);
             }
             if (more) {
 #pragma unroll

@@ -118,17 +118,37 @@ DCN_API int dcn_forward_algo(const void* x, const void* offset, const void* mask
                      int algo, void* stream);
 
 /*
- * dcn_forward_timeouts - bounded waits of the band kernel that ran out.
+ * dcn_device_flags - the per-device status word of the library's kernels.
  *
- * Every wait of the band kernel on its pipeline barriers gives up after about
- * two seconds; one that does sets a word on the current device, and its CTA
- * stops (the output of that call is then incomplete).  This returns that
- * word (0: no wait has ever run out on this device since the library was
- * loaded), reading it with a synchronous copy: it waits for the device's
- * preceding work.  No counterpart on the pages: a guard of this library's
- * own pipeline.  Returns DCN_ERR_CUDA if the read fails.
+ * Bits (sticky until reset):
+ *   DCN_FLAG_WAIT_TIMEOUT   a bounded wait of a band kernel's pipeline gave up
+ *                           after about two seconds; its CTA stopped, so the
+ *                           output of that call is incomplete;
+ *   DCN_FLAG_OUT_OF_BOUNDS  (debug library only) a kernel computed a gather,
+ *                           shared-memory or store address outside its buffer;
+ *                           the access was skipped (a load read zeros);
+ *   DCN_FLAG_BAD_LEVELS     (debug library only) an MSDA level table that is not
+ *                           a gap-free, in-order list of positive shapes; the
+ *                           call then reads no value rows.
+ * Returns the word of the current device and clears it when reset != 0. The
+ * read is a synchronous copy: it waits for the device's preceding work.
+ * No counterpart on the pages: a guard of this library's own kernels.
+ * Returns DCN_ERR_CUDA if the read fails.
  */
-DCN_API int dcn_forward_timeouts(void);
+#define DCN_FLAG_WAIT_TIMEOUT 1
+#define DCN_FLAG_OUT_OF_BOUNDS 2
+#define DCN_FLAG_BAD_LEVELS 4
+
+DCN_API int dcn_device_flags(int reset);
+
+/*
+ * dcn_debug_checks - 1 when this library was built with the device-side
+ * checks (the debug library, libdcn_b200_debug.so: every DCN and MSDA forward
+ * gather and store address is checked against its buffer, and the MSDA level
+ * table on the device), else 0. The debug library has the same interface and
+ * the same results; it is slower.
+ */
+DCN_API int dcn_debug_checks(void);
 
 /*
  * msda_forward - multi-scale deformable attention core, forward.

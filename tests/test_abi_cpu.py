@@ -290,3 +290,14 @@ def test_dynconv_validation(lib, change, status):
     before = dcnb.dcn_launch_count()
     assert call_dyn(lib, **change) == status
     assert dcnb.dcn_launch_count() == before
+
+
+def test_debug_library_exports_the_forward_and_status_calls(lib):
+    dbg = dcnb.debug_library()
+    for name in dcnb._binding.DEBUG_SYMBOLS:
+        assert hasattr(dbg, name), name
+    assert dcnb.dcn_debug_checks(dbg) == 1
+    assert dcnb.dcn_debug_checks() == 0
+    # host-side validation is the same code in both libraries
+    assert dbg.dcn_forward_algo(X, OFF, MASK, OUT, 2, 8, 8, 15, 4, 3, 3, 1, 1, 1, 0, F16, 0,
+                                None) == dcnb.DCN_ERR_INVALID_ARG

@@ -138,4 +138,4 @@ def test_band_output_guard_bands_untouched():
 def test_band_no_wait_ran_out():
     """Runs last in this file: no bounded wait of the band kernel's pipeline
     has given up in any of the calls above."""
-    assert dcnb.dcn_forward_timeouts() == 0
+    assert dcnb.dcn_device_flags() & dcnb.DCN_FLAG_WAIT_TIMEOUT == 0

@@ -98,7 +98,7 @@ def test_fused_band_kernel_rejects_other_shapes():
 
 
 def test_fused_no_wait_ran_out():
-    assert dcnb.dcn_forward_timeouts() == 0
+    assert dcnb.dcn_device_flags() & dcnb.DCN_FLAG_WAIT_TIMEOUT == 0
 
 
 def test_fused_without_bias_and_one_launch():
