@@ -337,7 +337,9 @@ int msda_backward(const void* value, const int64_t* spatial_shapes, const int64_
     const int tpi = D / cpt;
     if (tpi > 32) return DCN_ERR_UNSUPPORTED;
     const int run_items = 32 / tpi;
-    const int slice = dcnb::msda_bwd_slice(run_items, LK, es).total();
+    const int loc_stride = staged_row_stride(run_items, LK * 2, 2, es);
+    const int w_stride = staged_row_stride(run_items, LK, 1, es);
+    const int slice = dcnb::msda_bwd_slice(run_items, loc_stride, w_stride, es).total();
     if (slice > kMaxBwdSliceBytes || slice * dcnb::kMsdaWarps > kMaxBwdSmemBytes)
         return DCN_ERR_UNSUPPORTED;
 
@@ -360,6 +362,8 @@ int msda_backward(const void* value, const int64_t* spatial_shapes, const int64_
     a.total_items = (int)items;
     a.num_runs = (int)((items + run_items - 1) / run_items);
     a.stage_elems = run_items * LK;
+    a.loc_stride = loc_stride;
+    a.w_stride = w_stride;
     a.div_M = make_div((uint32_t)M);
     a.div_Lq = make_div((uint32_t)(Lq > 0 ? Lq : 1));
     a.div_tpi = make_div((uint32_t)tpi);

@@ -191,6 +191,39 @@ TileShape choose_tile(int N, int Ho, int runs, int kernel_extent, int sms, int c
     return best;
 }
 
+int staged_row_stride(int items, int row_elems, int read_elems, int es) {
+    const int row_bytes = (row_elems * es + 15) & ~15;
+    const int read_bytes = read_elems * es;
+    int best_stride = row_bytes, best_worst = 1 << 30;
+    for (int pad = 0; pad < 128; pad += 16) {
+        const int stride = row_bytes + pad;
+        int worst = 0;
+        for (int off = 0; off + read_bytes <= row_elems * es && worst < best_worst;
+             off += read_bytes) {
+            // distinct 4-byte words per bank among the items' reads at `off`
+            int words[32][32];
+            int count[32] = {0};
+            for (int i = 0; i < items && i < 32; ++i) {
+                const int first = (i * stride + off) >> 2;
+                const int last = (i * stride + off + read_bytes - 1) >> 2;
+                for (int wd = first; wd <= last; ++wd) {
+                    const int bank = wd & 31;
+                    bool seen = false;
+                    for (int j = 0; j < count[bank]; ++j) seen = seen || words[bank][j] == wd;
+                    if (!seen && count[bank] < 32) words[bank][count[bank]++] = wd;
+                }
+            }
+            for (int b = 0; b < 32; ++b) worst = std::max(worst, count[b]);
+        }
+        if (worst < best_worst) {
+            best_worst = worst;
+            best_stride = stride;
+        }
+        if (best_worst <= 1) break;
+    }
+    return best_stride / es;
+}
+
 }  // namespace dcnb_abi
 
 using namespace dcnb_abi;

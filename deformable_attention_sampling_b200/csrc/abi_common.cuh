@@ -127,16 +127,25 @@ struct TileShape {
 TileShape choose_tile(int N, int Ho, int runs, int kernel_extent, int sms, int cap,
                       int warps_by_regs);
 
+// Item stride, in elements, of a warp's staged slice in shared memory: the
+// run's `items` rows of `row_elems` elements (`es` bytes each) are copied
+// from consecutive global rows, and at every step each item reads
+// `read_elems` elements at the same offset of its row.  The stride is the row
+// rounded up to 16 bytes plus the multiple of 16 bytes that leaves the
+// fewest of those reads in one of the 32 four-byte banks (rows of a power of
+// two bytes would put every item in the same bank).
+int staged_row_stride(int items, int row_elems, int read_elems, int es);
+
+// Device address of the kernels' status word (DCN_FLAG_* bits) on the current
+// device (looked up once per device), or null.
+unsigned int* device_flags_word();
+
 // A 2-D tensor map over a row-major matrix of 16-bit elements (`inner`
 // elements per row, `outer` rows, rows `row_bytes` apart) for tile loads of
 // box_inner x box_outer elements with the 128-byte swizzle; out-of-range box
 // elements read as zero.  The encoder comes from the driver through the
 // runtime's entry-point query (no link-time dependency on libcuda).  False on
 // any error.
-// Device address of the kernels' status word (DCN_FLAG_* bits) on the current
-// device (looked up once per device), or null.
-unsigned int* device_flags_word();
-
 bool encode_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner,
                     uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 

@@ -79,7 +79,9 @@ static int msda_launch(const void* value, const int64_t* spatial_shapes,
     // per-warp shared slice for the run's locations and weights; unstaged when
     // the CTA's slices would not fit in the default shared-memory window
     int stage_elems = run_items * LK;
-    const int slice = ((2 * stage_elems * es + 15) & ~15) + ((stage_elems * es + 15) & ~15);
+    const int loc_stride = staged_row_stride(run_items, LK * 2, 2, es);
+    const int w_stride = staged_row_stride(run_items, LK, 1, es);
+    const int slice = run_items * (loc_stride + w_stride) * es;
     int smem = slice * dcnb::kMsdaWarps;
     if (smem > kMaxStageBytes) {
         stage_elems = 0;
@@ -103,6 +105,8 @@ static int msda_launch(const void* value, const int64_t* spatial_shapes,
     a.total_items = (int)items;
     a.num_runs = (int)((items + run_items - 1) / run_items);
     a.stage_elems = stage_elems;
+    a.loc_stride = loc_stride;
+    a.w_stride = w_stride;
     a.div_M = make_div((uint32_t)M);
     a.div_Lq = make_div((uint32_t)Lq);
     a.div_tpi = make_div((uint32_t)tpi);

@@ -71,16 +71,18 @@ __device__ __forceinline__ MsdaBwdTap msda_bwd_tap(const int (*lvl)[3], long lon
 }
 
 // Byte sizes of one warp's shared slice: staged locations and weights, then
-// grad_loc and grad_attn of the run (each part a multiple of 16 bytes).
+// grad_loc and grad_attn of the run, item rows loc_stride / w_stride elements
+// apart (each a multiple of 16 bytes).
 struct MsdaBwdSlice {
     int loc, attn;
     __host__ __device__ int total() const { return 2 * (loc + attn); }
 };
 
-__host__ __device__ inline MsdaBwdSlice msda_bwd_slice(int run_items, int LK, int es) {
+__host__ __device__ inline MsdaBwdSlice msda_bwd_slice(int run_items, int loc_stride,
+                                                       int w_stride, int es) {
     MsdaBwdSlice s;
-    s.loc = (2 * run_items * LK * es + 15) & ~15;
-    s.attn = (run_items * LK * es + 15) & ~15;
+    s.loc = run_items * loc_stride * es;
+    s.attn = run_items * w_stride * es;
     return s;
 }
 
@@ -100,7 +102,7 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_bwd_kernel(const MsdaBwd
     const int LK = L * K;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const MsdaBwdSlice sl = msda_bwd_slice(a.run_items, LK, es);
+    const MsdaBwdSlice sl = msda_bwd_slice(a.run_items, a.loc_stride, a.w_stride, es);
     unsigned char* my = smem + warp * sl.total();
     T* s_loc = reinterpret_cast<T*>(my);
     T* s_w = reinterpret_cast<T*>(my + sl.loc);
@@ -125,17 +127,21 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_bwd_kernel(const MsdaBwd
         const int item0 = run * a.run_items;
         const int nitems = min(a.run_items, a.total_items - item0);
         __syncwarp();
-        msda_warp_stage(s_loc, static_cast<const T*>(a.loc) + (long long)item0 * LK * 2,
-                        nitems * LK * 2, lane);
-        msda_warp_stage(s_w, static_cast<const T*>(a.attn) + (long long)item0 * LK, nitems * LK,
-                        lane);
+        msda_stage_rows<T, true>(
+            s_loc, a.loc_stride,
+            const_cast<T*>(static_cast<const T*>(a.loc)) + (long long)item0 * LK * 2, LK * 2,
+            nitems, lane);
+        msda_stage_rows<T, true>(
+            s_w, a.w_stride,
+            const_cast<T*>(static_cast<const T*>(a.attn)) + (long long)item0 * LK, LK, nitems,
+            lane);
         __syncwarp();
 
         // lanes without an item shadow item 0 with a zero upstream gradient
         const bool active = li_raw < nitems;
         const int li = active ? li_raw : 0;
-        const T* locp = s_loc + li * LK * 2;
-        const T* wp = s_w + li * LK;
+        const T* locp = s_loc + li * a.loc_stride;
+        const T* wp = s_w + li * a.w_stride;
         const int item = item0 + li;                  // (n * Lq + q) * M + h
         const int nq = (int)a.div_M.div((uint32_t)item);
         const int h = item - nq * a.M;
@@ -207,18 +213,19 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_bwd_kernel(const MsdaBwd
             da = item_sum(da, a.tpi, li_raw * a.tpi, chunk);
             db = item_sum(db, a.tpi, li_raw * a.tpi, chunk);
             if (active && chunk == 0) {
-                const int idx = li * LK + t;
-                s_gloc[2 * idx] = Elem<T>::from(A * cur.Wl * da);
-                s_gloc[2 * idx + 1] = Elem<T>::from(A * cur.Hl * db);
-                s_gw[idx] = Elem<T>::from(gs);
+                s_gloc[li * a.loc_stride + 2 * t] = Elem<T>::from(A * cur.Wl * da);
+                s_gloc[li * a.loc_stride + 2 * t + 1] = Elem<T>::from(A * cur.Hl * db);
+                s_gw[li * a.w_stride + t] = Elem<T>::from(gs);
             }
             if (more) cur = nxt;
         }
         __syncwarp();
-        warp_stage_out(static_cast<T*>(b.grad_loc) + (long long)item0 * LK * 2, s_gloc,
-                       nitems * LK * 2, lane);
-        warp_stage_out(static_cast<T*>(b.grad_attn) + (long long)item0 * LK, s_gw, nitems * LK,
-                       lane);
+        msda_stage_rows<T, false>(s_gloc, a.loc_stride,
+                                  static_cast<T*>(b.grad_loc) + (long long)item0 * LK * 2,
+                                  LK * 2, nitems, lane);
+        msda_stage_rows<T, false>(s_gw, a.w_stride,
+                                  static_cast<T*>(b.grad_attn) + (long long)item0 * LK, LK,
+                                  nitems, lane);
     }
 }
 

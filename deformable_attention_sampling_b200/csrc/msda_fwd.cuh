@@ -50,6 +50,7 @@ struct MsdaArgs {
     int total_items;             // N * Lq * M
     int num_runs;                // ceil(total_items / run_items)
     int stage_elems;             // staged weights per warp (run_items * L * K); 0 = unstaged
+    int loc_stride, w_stride;    // item strides (elements) of the staged slices
     FastDiv div_M, div_Lq, div_tpi;
     const void* ref;             // reference variants: [N][Lq][2 or 4] in valid-image units
     const void* vr;              // [N][L][2] valid ratios (W_valid / W, H_valid / H) or null
@@ -133,29 +134,58 @@ __device__ __forceinline__ MsdaTap msda_corners(const int (*lvl)[3], long long p
     return t;
 }
 
-// Copy `elems` elements of T from global `src` to shared `dst` with the lanes
-// of one warp (the widest access the addresses and the size allow).
-template <typename T>
-__device__ __forceinline__ void msda_warp_stage(T* dst, const T* src, int elems, int lane) {
-    const int nbytes = elems * (int)sizeof(T);
-    const uintptr_t al = (uintptr_t)src | (uintptr_t)dst | (uintptr_t)nbytes;
+// Element of `es` bytes, moved as an integer.
+template <int ES>
+struct Word;
+template <>
+struct Word<4> {
+    using type = uint32_t;
+};
+template <>
+struct Word<2> {
+    using type = unsigned short;
+};
+
+// Copy `rows` rows of `row_elems` elements of T between consecutive rows in
+// global memory and shared rows `stride` elements apart, with the lanes of
+// one warp; 16-byte vectors when the addresses and sizes allow, else single
+// elements.  IN: global -> shared; otherwise shared -> global.
+template <typename T, bool IN>
+__device__ __forceinline__ void msda_stage_rows(T* shared, int stride, T* global, int row_elems,
+                                                int rows, int lane) {
+    constexpr int es = (int)sizeof(T);
+    const int row_bytes = row_elems * es;
+    const uintptr_t al = (uintptr_t)global | (uintptr_t)shared | (uintptr_t)row_bytes |
+                         (uintptr_t)(stride * es);
     if ((al & 15) == 0) {
-        const uint4* s = reinterpret_cast<const uint4*>(src);
-        uint4* d = reinterpret_cast<uint4*>(dst);
-        for (int i = lane; i < (nbytes >> 4); i += 32) {
-            uint4 x;
-            asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w) : "l"(s + i));
-            d[i] = x;
+        const int vpr = row_bytes >> 4;
+        const int svs = (stride * es) >> 4;
+        uint4* g = reinterpret_cast<uint4*>(global);
+        uint4* sh = reinterpret_cast<uint4*>(shared);
+        for (int i = lane; i < rows * vpr; i += 32) {
+            const int r = i / vpr;
+            const int si = r * svs + (i - r * vpr);
+            if constexpr (IN) {
+                uint4 x;
+                asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                    : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w) : "l"(g + i));
+                sh[si] = x;
+            } else {
+                g[i] = sh[si];
+            }
         }
-    } else if ((al & 3) == 0) {
-        const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
-        uint32_t* d = reinterpret_cast<uint32_t*>(dst);
-        for (int i = lane; i < (nbytes >> 2); i += 32) d[i] = __ldg(s + i);
     } else {
-        const unsigned short* s = reinterpret_cast<const unsigned short*>(src);
-        unsigned short* d = reinterpret_cast<unsigned short*>(dst);
-        for (int i = lane; i < (nbytes >> 1); i += 32) d[i] = __ldg(s + i);
+        using W = typename Word<es>::type;
+        W* g = reinterpret_cast<W*>(global);
+        W* sh = reinterpret_cast<W*>(shared);
+        for (int i = lane; i < rows * row_elems; i += 32) {
+            const int r = i / row_elems;
+            const int si = r * stride + (i - r * row_elems);
+            if constexpr (IN)
+                sh[si] = __ldg(g + i);
+            else
+                g[i] = sh[si];
+        }
     }
 }
 
@@ -179,8 +209,9 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArg
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const bool staged = a.stage_elems > 0;
-    const int loc_slice = ((2 * a.stage_elems * (int)sizeof(T)) + 15) & ~15;
-    const int slice = loc_slice + ((a.stage_elems * (int)sizeof(T) + 15) & ~15);
+    // item rows a.loc_stride / a.w_stride elements apart (multiples of 16 bytes)
+    const int loc_slice = a.run_items * a.loc_stride * (int)sizeof(T);
+    const int slice = loc_slice + a.run_items * a.w_stride * (int)sizeof(T);
     T* s_loc = reinterpret_cast<T*>(smem + warp * slice);
     T* s_w = reinterpret_cast<T*>(smem + warp * slice + loc_slice);
 
@@ -229,13 +260,17 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArg
         const T* wp;
         if (staged) {
             __syncwarp();
-            msda_warp_stage(s_loc, static_cast<const T*>(a.loc) + (long long)item0 * LK * 2,
-                            nitems * LK * 2, lane);
-            msda_warp_stage(s_w, static_cast<const T*>(a.attn) + (long long)item0 * LK,
-                            nitems * LK, lane);
+            msda_stage_rows<T, true>(
+                s_loc, a.loc_stride,
+                const_cast<T*>(static_cast<const T*>(a.loc)) + (long long)item0 * LK * 2, LK * 2,
+                nitems, lane);
+            msda_stage_rows<T, true>(
+                s_w, a.w_stride,
+                const_cast<T*>(static_cast<const T*>(a.attn)) + (long long)item0 * LK, LK,
+                nitems, lane);
             __syncwarp();
-            locp = s_loc + li * LK * 2;
-            wp = s_w + li * LK;
+            locp = s_loc + li * a.loc_stride;
+            wp = s_w + li * a.w_stride;
         } else {
             locp = static_cast<const T*>(a.loc) + (long long)(item0 + li) * LK * 2;
             wp = static_cast<const T*>(a.attn) + (long long)(item0 + li) * LK;
