@@ -123,7 +123,10 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_bwd_kernel(const MsdaBwd
     const int r_begin = (int)(((long long)a.num_runs * blockIdx.x) / gridDim.x);
     const int r_end = (int)(((long long)a.num_runs * (blockIdx.x + 1)) / gridDim.x);
 
-    for (int run = r_begin + warp; run < r_end; run += kMsdaWarps) {
+    // one contiguous sub-range of runs per warp (as in the forward)
+    const int w_begin = r_begin + (int)(((long long)(r_end - r_begin) * warp) / kMsdaWarps);
+    const int w_end = r_begin + (int)(((long long)(r_end - r_begin) * (warp + 1)) / kMsdaWarps);
+    for (int run = w_begin; run < w_end; ++run) {
         const int item0 = run * a.run_items;
         const int nitems = min(a.run_items, a.total_items - item0);
         __syncwarp();

@@ -196,8 +196,11 @@ __device__ __forceinline__ void msda_stage_rows(T* shared, int stride, T* global
 // reference of the query and the level's valid ratio r:
 //   point: x = (cx r) W + dx - 1/2                  (s = cx r + dx / W)
 //   box:   x = ((cx + dx w / (2K)) r) W - 1/2       (s = cx r + dx / K * w * r / 2)
+// Five CTAs (20 warps) per SM for the plain path, four for the reference
+// variants, whose double-precision location arithmetic needs the registers.
 template <typename T, int VB, int REF = 0>
-__global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArgs a) {
+__global__ void __launch_bounds__(kMsdaThreads, REF == 0 ? 5 : 4)
+    msda_fwd_kernel(const MsdaArgs a) {
     constexpr int CPT = VB / (int)sizeof(T);
     constexpr int NW = VB >= 4 ? VB / 4 : 1;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -249,11 +252,16 @@ __global__ void __launch_bounds__(kMsdaThreads, 4) msda_fwd_kernel(const MsdaArg
     const int chunk = lane - li * a.tpi;
     const long long pix_bytes = (long long)a.M * a.D * (int)sizeof(T);   // one value row
 
-    // contiguous, balanced range of runs for this CTA; its warps interleave
+    // contiguous, balanced range of runs for this CTA, split into one
+    // contiguous sub-range per warp: consecutive queries of one warp reuse
+    // each other's value rows through L1, while the CTA's warps, working far
+    // apart, do not queue on the same lines' misses at the same time
     const int r_begin = (int)(((long long)a.num_runs * blockIdx.x) / gridDim.x);
     const int r_end = (int)(((long long)a.num_runs * (blockIdx.x + 1)) / gridDim.x);
+    const int w_begin = r_begin + (int)(((long long)(r_end - r_begin) * warp) / kMsdaWarps);
+    const int w_end = r_begin + (int)(((long long)(r_end - r_begin) * (warp + 1)) / kMsdaWarps);
 
-    for (int run = r_begin + warp; run < r_end; run += kMsdaWarps) {
+    for (int run = w_begin; run < w_end; ++run) {
         const int item0 = run * a.run_items;
         const int nitems = min(a.run_items, a.total_items - item0);
         const T* locp;

@@ -168,6 +168,10 @@ class MsdaWorkload:
     dtype: str = "f32"
     offset_sigma: float = 2.0  # std of the pixel offsets at each level
     ref_dim: int = 0          # 2 / 4: reference points / boxes with valid ratios
+    # reference points of msda_inputs: "cell" puts each encoder query at its
+    # own cell centre (the query is that cell), "uniform" draws them ~U[0,1]^2;
+    # "" means "cell" for encoder-style queries (Lq = 0), else "uniform"
+    ref_points: str = ""
 
     @property
     def L(self):
@@ -229,9 +233,16 @@ WORKLOADS = {w.name: w for w in [
     # the 7 x 7 and 13 x 13 kernel sizes of the OverLoCK networks
     DynWorkload("contmix_f16_64x56x56x64_g4_k7", N=64, H=56, W=56, C=64, G=4, K=7),
     DynWorkload("contmix_f16_64x56x56x64_g4_k13", N=64, H=56, W=56, C=64, G=4, K=13),
-    # MSDeformAttn, four levels, encoder-style queries
+    # MSDeformAttn, four levels, encoder-style queries: one query per cell of
+    # every level, referenced at its own cell centre
     MsdaWorkload("msda_f32_2x4lvl_m8_d32_k4", N=2, M=8, D=32,
                  shapes=((100, 150), (50, 75), (25, 38), (13, 19)), K=4, dtype="f32"),
+    # the same queries with reference points drawn uniformly over the image:
+    # no two consecutive queries share a neighbourhood (a stress case for the
+    # gather path)
+    MsdaWorkload("msda_f32_2x4lvl_m8_d32_k4_uniformref", N=2, M=8, D=32,
+                 shapes=((100, 150), (50, 75), (25, 38), (13, 19)), K=4, dtype="f32",
+                 ref_points="uniform"),
     # the same levels as a decoder with 4-D box references, valid ratios and
     # 300 object queries per image
     MsdaWorkload("msda_f32_2x4lvl_m8_d32_k4_box300", N=2, M=8, D=32,
@@ -275,14 +286,35 @@ def level_start_index(shapes):
     return starts
 
 
+def msda_centres(shapes):
+    """Normalised centres (x, y) = ((j + 1/2) / W_l, (i + 1/2) / H_l) of every
+    cell of every level, in the row order of the concatenated value tensor."""
+    parts = []
+    for h, wd in shapes:
+        cx, cy = np.meshgrid((np.arange(wd) + 0.5) / wd, (np.arange(h) + 0.5) / h, indexing="xy")
+        parts.append(np.stack([cx, cy], axis=-1).reshape(-1, 2))
+    return np.concatenate(parts, axis=0)
+
+
 def msda_inputs(w, seed=0):
-    """value [N,S,M,D] ~ U[-1,1]; one reference point per (n, q) ~ U[0,1]^2 shared
-    by heads, levels and points; pixel offsets ~ N(0, sigma) per (m, l, k) divided
-    by (W_l, H_l); logits ~ N(0,1) normalised jointly over (l, k) per head."""
+    """value [N,S,M,D] ~ U[-1,1]; one reference point per (n, q) shared by heads,
+    levels and points: for encoder-style queries (one per cell, Lq = 0) the
+    centre of the query's own cell, normalised by its level ("Deformable
+    DETR": in the encoder a source cell centre is the reference), otherwise
+    ~ U[0,1]^2 (w.ref_points overrides); pixel offsets ~ N(0, sigma) per
+    (m, l, k) divided by (W_l, H_l); logits ~ N(0,1) normalised jointly over
+    (l, k) per head."""
     rng = np.random.default_rng(seed)
     Lq = w.queries
     value = rng.uniform(-1.0, 1.0, size=(w.N, w.S, w.M, w.D))
-    ref = rng.uniform(0.0, 1.0, size=(w.N, Lq, 2))
+    ref = rng.uniform(0.0, 1.0, size=(w.N, Lq, 2))   # drawn in every mode: same stream
+    mode = w.ref_points or ("cell" if not w.Lq else "uniform")
+    if mode == "cell":
+        if Lq != w.S:
+            raise ValueError("cell-centre references need one query per cell (Lq = 0)")
+        ref = np.broadcast_to(msda_centres(w.shapes)[None], (w.N, Lq, 2))
+    elif mode != "uniform":
+        raise ValueError(f"unknown reference-point mode {mode!r}")
     dp = rng.normal(0.0, w.offset_sigma, size=(w.N, Lq, w.M, w.L, w.K, 2))
     logits = rng.normal(0.0, 1.0, size=(w.N, Lq, w.M, w.L, w.K))
     size_wh = np.array([[wd, h] for h, wd in w.shapes], dtype=np.float64)  # [L, 2]
