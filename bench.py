@@ -388,8 +388,9 @@ class MsdaBwdRunner(MsdaRunner):
 
 
 class DynRunner:
-    """One step = one dynconv_forward call (the ContMix core)."""
+    """One step = one dynconv_forward_algo call (the ContMix core)."""
     kernel = "dynconv_fwd_kernel"
+    algo = 0     # DCN_ALGO_AUTO; set from --algo
 
     def __init__(self, w, seed, device):
         import deformable_attention_sampling_b200 as dcnb
@@ -408,12 +409,12 @@ class DynRunner:
     def launcher(self, s, stream):
         w, lib = self.w, self.lib
         args = (s["x"].data_ptr(), s["weights"].data_ptr(), s["out"].data_ptr(), w.N, w.H, w.W,
-                w.C, w.G, w.K, w.softmax_flag, self.code, stream)
+                w.C, w.G, w.K, w.softmax_flag, self.code, self.algo, stream)
 
         def go():
-            st = lib.dynconv_forward(*args)
+            st = lib.dynconv_forward_algo(*args)
             if st != 0:
-                raise self.dcnb.DcnError(st, "dynconv_forward")
+                raise self.dcnb.DcnError(st, "dynconv_forward_algo")
         return go
 
     def inputs_of(self, s):
@@ -688,7 +689,24 @@ def run_b200(args):
     backward = args.pass_ == "backward"
     runner = make_runner(w, seed=1000 + rank, device=device, backward=backward)
     band = False
-    if isinstance(runner, DcnRunner) and not backward:
+    dyn_algos = ("auto", "simt", "tensor")
+    if isinstance(runner, DynRunner) != (args.algo in dyn_algos[1:]) and args.algo != "auto":
+        raise ValueError(f"--algo {args.algo} does not apply to workload {w.name}")
+    if isinstance(runner, DynRunner):
+        runner.algo = dcnb.DYNCONV_ALGO_CODES[args.algo]
+        # which kernel the timed calls run: the tensor-core one where it applies
+        tensor = False
+        if args.algo != "simt":
+            probe = runner.alloc_set()
+            tensor = dcnb.library().dynconv_forward_algo(
+                probe["x"].data_ptr(), probe["weights"].data_ptr(), probe["out"].data_ptr(),
+                w.N, w.H, w.W, w.C, w.G, w.K, w.softmax_flag, runner.code,
+                dcnb.DCN_ALGO_TENSOR, int(torch.cuda.current_stream(device).cuda_stream)) == 0
+            torch.cuda.synchronize(device)
+            del probe
+        runner.kernel = ("dynconv_mma_kernel (mma.sync m16n8k16)" if tensor
+                         else "dynconv_fwd_kernel")
+    elif isinstance(runner, DcnRunner) and not backward:
         runner.algo = dcnb.ALGO_CODES[args.algo]
         # which kernel the timed calls run: the band kernel where it applies
         if args.algo != "gather":
@@ -959,8 +977,10 @@ def main():
     p.add_argument("--workload", default=gen.HEADLINE, choices=sorted(gen.WORKLOADS))
     p.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
                    help="time the forward call (default) or the backward call")
-    p.add_argument("--algo", default="auto", choices=["auto", "gather", "band"],
-                   help="DCN forward kernel (dcn_forward_algo); auto = dcn_forward")
+    p.add_argument("--algo", default="auto", choices=["auto", "gather", "band", "simt", "tensor"],
+                   help="the kernel: gather / band for the DCN forward (dcn_forward_algo), "
+                        "simt / tensor for the ContMix core (dynconv_forward_algo); "
+                        "auto = each call's default")
     args = p.parse_args()
     if args.warmup < 3:
         p.error("--warmup must be at least 3")

@@ -17,6 +17,9 @@ from ._binding import (  # noqa: F401
     DCN_ALGO_AUTO,
     DCN_ALGO_BAND,
     DCN_ALGO_GATHER,
+    DCN_ALGO_SIMT,
+    DCN_ALGO_TENSOR,
+    DYNCONV_ALGO_CODES,
     DCN_ERR_CUDA,
     DCN_ERR_INVALID_ARG,
     DCN_ERR_MISALIGNED,
@@ -52,6 +55,7 @@ from ._binding import (  # noqa: F401
     dtype_code,
     dynconv,
     dynconv_forward,
+    dynconv_forward_algo,
     library,
     msda,
     msda_backward,

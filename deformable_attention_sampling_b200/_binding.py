@@ -32,8 +32,12 @@ DEBUG_SYMBOLS = ("dcn_forward", "dcn_forward_algo", "dcnv4_fused_forward",
                  "dcn_launch_count", "dcn_device_flags", "dcn_debug_checks", "dcn_version")
 DCN_ALGO_AUTO = 0
 DCN_ALGO_GATHER = 1
+DCN_ALGO_SIMT = 1
 DCN_ALGO_BAND = 2
+DCN_ALGO_TENSOR = 3
 ALGO_CODES = {"auto": DCN_ALGO_AUTO, "gather": DCN_ALGO_GATHER, "band": DCN_ALGO_BAND}
+# dynconv_forward_algo's kernels
+DYNCONV_ALGO_CODES = {"auto": DCN_ALGO_AUTO, "simt": DCN_ALGO_SIMT, "tensor": DCN_ALGO_TENSOR}
 
 # every symbol include/dcn.h declares, with its ctypes signature
 _VP = ctypes.c_void_p
@@ -53,6 +57,7 @@ SIGNATURES = {
     "msda_backward_workspace_size": (_LL, [_I] * 5),
     "msda_backward": (_I, [_VP] * 10 + [_LL] + [_I] * 8 + [_VP]),
     "dynconv_forward": (_I, [_VP] * 3 + [_I] * 8 + [_VP]),
+    "dynconv_forward_algo": (_I, [_VP] * 3 + [_I] * 9 + [_VP]),
     "dcnv4_fused_forward": (_I, [_VP] * 4 + [_I] * 10 + [_VP]),
     "dcnv4_fused_forward_algo": (_I, [_VP] * 4 + [_I] * 11 + [_VP]),
     "dcn_output_size": (_I, [_I] * 5),
@@ -235,6 +240,14 @@ def dynconv_forward(x, weights, out, N, H, W, C, G, K, softmax_flag, dtype, stre
     _check(_load().dynconv_forward(_ptr(x), _ptr(weights), _ptr(out), N, H, W, C, G, K,
                                    softmax_flag, dtype, _stream(stream)),
            "dynconv_forward")
+
+
+def dynconv_forward_algo(x, weights, out, N, H, W, C, G, K, softmax_flag, dtype, algo,
+                         stream=None):
+    """C dynconv_forward_algo; raises DcnError on a non-OK status."""
+    _check(_load().dynconv_forward_algo(_ptr(x), _ptr(weights), _ptr(out), N, H, W, C, G, K,
+                                        softmax_flag, dtype, algo, _stream(stream)),
+           "dynconv_forward_algo")
 
 
 def msda_forward_points(value, spatial_shapes, level_start, reference, ref_dim, valid_ratios,
@@ -439,10 +452,11 @@ def msda_grad(value, spatial_shapes, level_start, sampling_loc, attn_w, grad_out
     return gv, gl, ga
 
 
-def dynconv(x, weights, K, softmax_flag=1, out=None, stream=None):
-    """dynconv_forward (the ContMix core) on torch CUDA tensors.
+def dynconv(x, weights, K, softmax_flag=1, out=None, stream=None, algo="auto"):
+    """dynconv_forward_algo (the ContMix core) on torch CUDA tensors.
 
     x [N, H, W, C], weights [N, H, W, G, K*K] (tap ky * K + kx), one dtype.
+    algo: "auto" (the tensor-core kernel where it applies), "tensor" or "simt".
     """
     import torch
     _require(x.dim() == 4 and weights.dim() == 5, "expected x [N,H,W,C], weights [N,H,W,G,K*K]")
@@ -456,7 +470,9 @@ def dynconv(x, weights, K, softmax_flag=1, out=None, stream=None):
         out = torch.empty_like(x)
     _require(tuple(out.shape) == (N, H, W, C) and out.dtype == x.dtype and out.is_contiguous(),
              "out has the wrong shape, dtype or layout")
-    dynconv_forward(x, weights, out, N, H, W, C, G, K, softmax_flag, dtype_code(x), stream)
+    _require(algo in DYNCONV_ALGO_CODES, f"algo must be one of {sorted(DYNCONV_ALGO_CODES)}")
+    dynconv_forward_algo(x, weights, out, N, H, W, C, G, K, softmax_flag, dtype_code(x),
+                         DYNCONV_ALGO_CODES[algo], stream)
     return out
 
 

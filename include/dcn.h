@@ -110,7 +110,13 @@ DCN_API int dcn_forward(const void* x, const void* offset, const void* mask, voi
  * last bit where the order of the float32 additions differs.
  * Errors: as dcn_forward, plus DCN_ERR_INVALID_ARG for an unknown `algo`.
  */
-typedef enum { DCN_ALGO_AUTO = 0, DCN_ALGO_GATHER = 1, DCN_ALGO_BAND = 2 } dcn_algo_t;
+typedef enum {
+    DCN_ALGO_AUTO = 0,
+    DCN_ALGO_GATHER = 1,
+    DCN_ALGO_SIMT = 1,      /* dynconv_forward_algo: the CUDA-core (FFMA) kernel */
+    DCN_ALGO_BAND = 2,
+    DCN_ALGO_TENSOR = 3     /* dynconv_forward_algo: the tensor-core kernel */
+} dcn_algo_t;
 
 DCN_API int dcn_forward_algo(const void* x, const void* offset, const void* mask, void* out,
                      int N, int H, int W, int C, int G, int kh, int kw,
@@ -438,6 +444,31 @@ DCN_API int msda_backward(const void* value, const int64_t* spatial_shapes,
  */
 DCN_API int dynconv_forward(const void* x, const void* weights, void* out, int N, int H,
                  int W, int C, int G, int K, int softmax_flag, int dtype, void* stream);
+
+/*
+ * dynconv_forward_algo - dynconv_forward with the kernel chosen by `algo`.
+ *
+ *   DCN_ALGO_TENSOR  each kernel row of 16 consecutive outputs as a banded
+ *                    16 x 32 matrix (the locations' K numbers) times the
+ *                    window row (32 columns x 16 channels) on the tensor cores
+ *                    (mma.sync m16n8k16, float32 accumulation); the softmaxed
+ *                    numbers enter as a 16-bit high part plus the 16-bit
+ *                    rounding of the remainder.  Only for f16 / bf16 data and
+ *                    K = 7 or 13: DCN_ERR_UNSUPPORTED otherwise.  A non-finite
+ *                    x value inside the 32-column window of a 16-output block
+ *                    makes all of that block's outputs of the row non-finite
+ *                    (the band's zeros multiply it), where the definition
+ *                    leaves outputs that do not reach it unaffected.
+ *   DCN_ALGO_SIMT    (= DCN_ALGO_GATHER) the CUDA-core kernel: float32 FMAs
+ *                    over the staged window, any dtype and odd K <= 31.
+ *   DCN_ALGO_AUTO    the tensor-core kernel where it applies, else the CUDA-core one.
+ * The two kernels add the same products in different orders; their outputs
+ * may differ in the last bit.
+ * Errors: as dynconv_forward, plus DCN_ERR_INVALID_ARG for an unknown `algo`.
+ */
+DCN_API int dynconv_forward_algo(const void* x, const void* weights, void* out, int N, int H,
+                 int W, int C, int G, int K, int softmax_flag, int dtype, int algo,
+                 void* stream);
 
 /* Output size of the deformable window: (in + 2 pad - dil (k - 1) - 1) / stride + 1,
  * or a value <= 0 when the window does not fit. */

@@ -292,6 +292,34 @@ def test_dynconv_validation(lib, change, status):
     assert dcnb.dcn_launch_count() == before
 
 
+@pytest.mark.parametrize("algo", [dcnb.DCN_ALGO_SIMT, dcnb.DCN_ALGO_TENSOR])
+@pytest.mark.parametrize("change,status", [
+    (dict(dtype=5), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(K=4), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(x=None), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(out=X), dcnb.DCN_ERR_INVALID_ARG),
+    (dict(out=OUT + 16), dcnb.DCN_ERR_MISALIGNED),
+    (dict(N=0), dcnb.DCN_OK),
+])
+def test_dynconv_forward_algo_validation(lib, algo, change, status):
+    args = dict(x=X, w=OFF, out=OUT, N=2, H=8, W=8, C=32, G=2, K=7, softmax_flag=1, dtype=F16)
+    args.update(change)
+    a = args
+    before = dcnb.dcn_launch_count()
+    assert lib.dynconv_forward_algo(a["x"], a["w"], a["out"], a["N"], a["H"], a["W"], a["C"],
+                                    a["G"], a["K"], a["softmax_flag"], a["dtype"], algo,
+                                    None) == status
+    assert dcnb.dcn_launch_count() == before
+
+
+@pytest.mark.parametrize("algo", [-1, 2, 4])
+def test_dynconv_forward_algo_rejects_unknown_kernels(lib, algo):
+    before = dcnb.dcn_launch_count()
+    assert lib.dynconv_forward_algo(X, OFF, OUT, 2, 8, 8, 32, 2, 7, 1, F16, algo,
+                                    None) == dcnb.DCN_ERR_INVALID_ARG
+    assert dcnb.dcn_launch_count() == before
+
+
 def test_debug_library_exports_the_forward_and_status_calls(lib):
     dbg = dcnb.debug_library()
     for name in dcnb._binding.DEBUG_SYMBOLS:

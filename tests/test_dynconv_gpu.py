@@ -16,8 +16,8 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def run(inp, w):
-    out = dcnb.dynconv(inp["x"].to(DEV), inp["weights"].to(DEV), w.K, w.softmax_flag)
+def run(inp, w, algo="auto"):
+    out = dcnb.dynconv(inp["x"].to(DEV), inp["weights"].to(DEV), w.K, w.softmax_flag, algo=algo)
     torch.cuda.synchronize()
     return out
 
@@ -30,13 +30,62 @@ def ref(inp, w, n=None):
 DYN_WORKLOADS = [n for n, w in gen.WORKLOADS.items() if isinstance(w, gen.DynWorkload)]
 
 
+@pytest.mark.parametrize("algo", ["tensor", "simt"])
 @pytest.mark.parametrize("name", DYN_WORKLOADS)
-def test_dynconv_workload_full_size(name):
+def test_dynconv_workload_full_size(name, algo):
     w = gen.WORKLOADS[name]
     inp = gen.dynconv_inputs(w, seed=0)
-    out = run(inp, w)
+    out = run(inp, w, algo)
     for n in sorted({0, w.N // 2, w.N - 1}):
-        compare(out[n:n + 1], ref(inp, w, n), f"{name} image {n}")
+        compare(out[n:n + 1], ref(inp, w, n), f"{name} {algo} image {n}")
+
+
+TENSOR_SMALL = [
+    # N, H, W, C, G, K, dtype, softmax: the tensor-core kernel (16-bit, K = 7 or 13)
+    (1, 1, 1, 16, 1, 7, "f16", 1),         # one pixel: every tap but the centre is padding
+    (2, 9, 17, 32, 2, 7, "f16", 1),        # second 16-column block holds one column
+    (1, 8, 32, 64, 4, 13, "bf16", 1),      # exactly one tile
+    (1, 19, 70, 16, 1, 13, "f16", 0),      # weights as given; ragged rows and columns
+    (2, 13, 40, 64, 2, 13, "bf16", 1),     # D = 32: two 16-channel chunks per group
+    (1, 3, 5, 48, 3, 13, "f16", 1),        # window wider and taller than the map
+    (3, 11, 45, 32, 2, 7, "bf16", 0),
+]
+
+
+@pytest.mark.parametrize("case", TENSOR_SMALL, ids=[f"tc{i}" for i in range(len(TENSOR_SMALL))])
+def test_dynconv_tensor_small_shapes(case):
+    N, H, W, C, G, K, dt, sm = case
+    w = gen.DynWorkload("tc", N=N, H=H, W=W, C=C, G=G, K=K, dtype=dt, softmax_flag=sm)
+    inp = gen.dynconv_inputs(w, seed=11)
+    expect = ref(inp, w)
+    tc = run(inp, w, "tensor")
+    compare(tc, expect, f"{case} tensor")
+    compare(run(inp, w, "simt"), expect, f"{case} simt")
+    assert torch.equal(run(inp, w, "auto"), tc), "auto takes the tensor-core kernel"
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_dynconv_tensor_large_logits(dt):
+    """Logits far from 0 and rising along the rows: the running maximum
+    grows from one kernel row to the next, so the accumulators are rescaled."""
+    w = gen.DynWorkload("big", N=1, H=12, W=35, C=32, G=2, K=13, dtype=dt)
+    inp = gen.dynconv_inputs(w, seed=6)
+    ramp = torch.arange(13, dtype=torch.float64).repeat_interleave(13) * 3.0
+    inp["weights"] = (inp["weights"].double() * 20.0 + 40.0 + ramp).to(inp["weights"].dtype)
+    compare(run(inp, w, "tensor"), ref(inp, w), f"large logits {dt}")
+
+
+def test_dynconv_tensor_rejects_what_it_does_not_cover():
+    for dt, K in (("f32", 7), ("f16", 5), ("bf16", 9)):
+        C = 16 if dt != "f32" else 8
+        w = gen.DynWorkload("rej", N=1, H=6, W=9, C=C, G=1, K=K, dtype=dt)
+        inp = gen.dynconv_inputs(w, seed=2)
+        with pytest.raises(dcnb.DcnError) as e:
+            run(inp, w, "tensor")
+        assert e.value.status == dcnb.DCN_ERR_UNSUPPORTED
+        compare(run(inp, w, "auto"), ref(inp, w), f"auto falls back ({dt}, K={K})")
+    with pytest.raises(ValueError):
+        run(inp, w, "band")
 
 
 SMALL = [
