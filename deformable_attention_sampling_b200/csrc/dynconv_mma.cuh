@@ -60,13 +60,15 @@ __host__ __device__ inline int mma_tile_offset(int bb, int s, int part) {
     return ((bb * 2 + s) * 2 + part) * kMmaTileBytes + bb * kMmaBlockPad;
 }
 
-// 4-byte words of a location's slot for one kernel row in the raw buffer:
-// its K numbers from the 4-byte word holding the first, rounded up to an odd
-// count, so that 32 lanes reading word k of their slots hit 32 banks.
-__host__ __device__ inline int dyn_mma_slot_words(int K) {
-    const int w = (2 * K + 2 + 3) / 4;
-    return w | 1;
+// 8-byte units of a location's slot for one kernel row in the raw buffer:
+// its K numbers from the 8-byte unit holding the first, rounded up to an odd
+// count, so that the 8-byte loads of 16 lanes (one wavefront) hit distinct
+// bank pairs.
+__host__ __device__ inline int dyn_mma_slot_units(int K) {
+    const int u = (2 * K + 6 + 7) / 8;
+    return u | 1;
 }
+__host__ __device__ inline int dyn_mma_slot_words(int K) { return 2 * dyn_mma_slot_units(K); }
 
 // Byte offset of element (row i, column jj) of a 16 x 16 tile of 16-bit
 // values: rows of 32 bytes, the two 16-byte halves of rows 4-7 and 12-15
@@ -152,10 +154,16 @@ __host__ __device__ inline int dyn_mma_smem(int K) {
            kMmaRows * kMmaWarpBytes;
 }
 
-// 4-byte asynchronous global -> shared copy of src_bytes (0..4) bytes, zero-filled.
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(dst), "l"(src),
+// 8-byte asynchronous global -> shared copy of src_bytes (0..8) bytes, zero-filled.
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" :: "r"(dst), "l"(src),
                  "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+    return v;
 }
 
 template <typename T, bool SOFTMAX, int K>
@@ -220,7 +228,7 @@ __global__ void __launch_bounds__(kMmaThreads, 2) dynconv_mma_kernel(const DynAr
     auto in_map = [&](int row, int col) { return y0 + row < a.H && x0 + col < a.W; };
     // Each thread copies and reads the numbers of its own location (warp, lane)
     // only, so the raw buffers need no barrier: kernel row ky goes to buffer
-    // ky & 1 as 4-byte words from the one holding the row's first number, the
+    // ky & 1 as 8-byte units from the one holding the row's first number, the
     // last clipped to the row's end.
     const bool mine = in_map(warp, lane);
     const char* my_w = reinterpret_cast<const char*>(wt + warp * w_row + lane * w_col);
@@ -230,18 +238,18 @@ __global__ void __launch_bounds__(kMmaThreads, 2) dynconv_mma_kernel(const DynAr
         if (mine) {
             const char* first = my_w + ky * K * es;
             const char* last = first + K * es;
-            const char* w4 = reinterpret_cast<const char*>((uintptr_t)first & ~(uintptr_t)3);
+            const char* u8 = reinterpret_cast<const char*>((uintptr_t)first & ~(uintptr_t)7);
             uint32_t dst = my_slot + (uint32_t)((ky & 1) * NP * SW * 4);
-            for (; w4 < last; w4 += 4, dst += 4) {
-                const long long left = last - w4;
-                cp_async4(dst, w4, left >= 4 ? 4u : (uint32_t)left);
+            for (; u8 < last; u8 += 8, dst += 8) {
+                const long long left = last - u8;
+                cp_async8(dst, u8, left >= 8 ? 8u : (uint32_t)left);
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
     // ---- softmax role: this lane's location (warp, lane) = block bb, row i ----
-    const int skew = (int)((uintptr_t)my_w & 3);
+    const int skew = (int)((uintptr_t)my_w & 7);
     const int bb_own = lane >> 4, i_own = lane & 15;
     uint32_t waddr[NWORD];   // shared address of band word k in the high tile
 #pragma unroll
@@ -295,14 +303,27 @@ __global__ void __launch_bounds__(kMmaThreads, 2) dynconv_mma_kernel(const DynAr
         e[2 * NWORD - 1] = 0.f;
         float sc = 1.f;
         if (mine) {
-            // the row's numbers start at half-word (skew + ky K es) / 2 & 1 of the slot:
-            // realign the word pairs, then widen
-            const uint32_t* zw = raw + ((ky & 1) * NP + warp * kMmaCols + lane) * SW;
-            const uint32_t al = (((skew + ky * K * es) & 3) != 0) ? 0x5432u : 0x3210u;
+            // the row's numbers start at byte o = (skew + ky K es) & 7 of the slot:
+            // load the slot, drop o / 4 words, realign the half-word pairs, widen
+            constexpr int NU = (2 * K + 6 + 7) / 8 | 1;   // = dyn_mma_slot_units(K)
+            const int o = (skew + ky * K * es) & 7;
+            const uint32_t zs = my_slot + (uint32_t)((ky & 1) * NP * SW * 4);
+            uint32_t wv[2 * NU];
+#pragma unroll
+            for (int u = 0; u < NU; ++u) {
+                const uint2 v = lds64(zs + 8 * u);
+                wv[2 * u] = v.x;
+                wv[2 * u + 1] = v.y;
+            }
+            const bool wshift = o >= 4;
+            const uint32_t al = (o & 2) ? 0x5432u : 0x3210u;
+            uint32_t wa[NWORD + 1];
+#pragma unroll
+            for (int k = 0; k <= NWORD; ++k) wa[k] = wshift ? wv[k + 1] : wv[k];
             float z[2 * NWORD];
 #pragma unroll
             for (int k = 0; k < NWORD; ++k) {
-                const float2 f = Ops::unpack(__byte_perm(zw[k], zw[k + 1], al));
+                const float2 f = Ops::unpack(__byte_perm(wa[k], wa[k + 1], al));
                 z[2 * k] = f.x;
                 z[2 * k + 1] = f.y;
             }
