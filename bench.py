@@ -51,8 +51,8 @@ SMEM_BYTES_PER_CLK = 128.0
 # dram__bytes_write.sum per launch, headline workload), with the hash of the
 # files the headline launch is built from; reported as null once they change.
 NCU_TRAFFIC = {
-    "source_sha256": "903eb45612d69b1b54e3254a75f26395c21cfcaf45eb8dc857a067e95c12028a",
-    "bytes_per_launch": 69523456 + 4337408,   # DRAM read + write, one headline launch
+    "source_sha256": "802729f0aa2721a26ffc6402658e360962d75eeb466464c78aaf784b6895bbfc",
+    "bytes_per_launch": 69676032 + 3020800,   # DRAM read + write, one headline launch
 }
 
 # What the headline dcn_forward launch is built from: its device code and the
