@@ -20,16 +20,17 @@
 // as the column-major B operand.  These operands are assembled per warp in
 // registers and shared memory, which is why this path uses the warp-level
 // mma.sync: a tcgen05 product would read A from shared memory or TMEM at
-// 128 rows x 32 columns per k-range, four tenths of it zeros, and for N = 16
+// 128 rows x 32 columns per k-range, six tenths of it zeros, and for N = 16
 // channels those operand reads, not the arithmetic, would set its time.
 //
 // Work decomposition (one CTA = 8 output rows x 32 columns of one group and
 // one 16-channel chunk; 8 warps):
 //   warp  = one output row, as two blocks of 16 columns;
-//   lane  = one location (column) of the row for the softmax: it reads its
-//           raw numbers of kernel row ky, updates its running maximum and
-//           sum (online softmax, as the SIMT kernel), and writes its band of
-//           A (high and low parts) for both k-steps;
+//   lane  = one location (column) of the row for the softmax: it copies its
+//           own numbers of kernel row ky + 1 into its own slot (8-byte
+//           cp.async, no barrier) while it reads row ky, updates its running
+//           maximum and sum (online softmax, as the SIMT kernel), and writes
+//           its band of A (high and low parts) for both k-steps;
 //   mma   = per block and k-step: A (ldmatrix.x4, high and low), B
 //           (ldmatrix.x4.trans: 16 window columns x 16 channels), four
 //           m16n8k16 products into float32 accumulators (16 per lane).
