@@ -862,12 +862,12 @@ def run_b200(args):
     if pool is not None:
         pool.close()
         pool.join()
-        if backward:
-            result["pass"] = "backward"
-            result["roofline"]["note"] = (
-                "timed over the whole dcn_backward / msda_backward call (zero fill, gradient "
-                "kernel, rounding); algorithmic bytes = inputs + grad_out read, three "
-                "gradients written once, no float32 accumulator traffic")
+    if result is not None and backward:
+        result["pass"] = "backward"
+        result["roofline"]["note"] = (
+            "timed over the whole dcn_backward / msda_backward call (zero fill, gradient "
+            "kernel, rounding); algorithmic bytes = inputs + grad_out read, three "
+            "gradients written once, no float32 accumulator traffic")
     if world > 1:
         import torch.distributed as dist
         dist.barrier(device_ids=[device.index])
