@@ -1,5 +1,6 @@
-"""Seeded random small shapes for every forward entry point, each checked
-element by element against the float64 oracle (tests/parity.py tolerances).
+"""Seeded random small shapes for every forward entry point and the two
+backward calls, each checked element by element against the float64 oracle
+(tests/parity.py tolerances).
 
 The shapes are drawn once from a fixed generator, so the test set is the same
 on every run. They cover the kernels' dispatch decisions between them:
@@ -107,3 +108,36 @@ def test_dynconv_random_shapes(case):
     torch.cuda.synchronize()
     ref = oracle.dynconv_forward_ref(inp["x"], inp["weights"], d.K, d.softmax_flag)
     compare(out, ref, str(case))
+
+
+# ------------------------------------------------------------------ backward
+
+@pytest.mark.parametrize("case", _dcn_cases(count=10, seed=4242), ids=lambda c: "dcnb_" + "_".join(
+    f"{k}{v}" for k, v in c.items() if k in ("N", "H", "W", "C", "G", "kh", "stride", "dtype")))
+def test_dcn_backward_random_shapes(case):
+    w = gen.DcnWorkload("rand", **case)
+    inp = gen.dcn_inputs(w, seed=6)
+    go = gen.grad_out((w.N, w.Ho, w.Wo, w.C), w.dtype, seed=6)
+    got = dcnb.dcn_grad(inp["x"].to(DEV), inp["offset"].to(DEV), inp["mask"].to(DEV),
+                        go.to(DEV), w.kh, w.kw, w.stride, w.pad, w.dil, w.softmax_flag)
+    torch.cuda.synchronize()
+    ref = oracle.dcn_backward_ref(inp["x"], inp["offset"], inp["mask"], go, w.kh, w.kw,
+                                  w.stride, w.pad, w.dil, w.softmax_flag)
+    for name, g, r in zip(("grad_x", "grad_offset", "grad_mask"), got, ref):
+        compare(g, r, f"{case} {name}")
+
+
+@pytest.mark.parametrize("case", _msda_cases(count=6, seed=99), ids=lambda c: "msdab_" + "_".join(
+    f"{k}{v}" for k, v in c.items() if k in ("N", "M", "D", "K", "Lq", "dtype")))
+def test_msda_backward_random_shapes(case):
+    m = gen.MsdaWorkload("rand", **case)
+    inp = gen.msda_inputs(m, seed=10)
+    go = gen.grad_out((m.N, m.queries, m.M * m.D), m.dtype, seed=10)
+    got = dcnb.msda_grad(inp["value"].to(DEV), inp["spatial_shapes"].to(DEV),
+                         inp["level_start"].to(DEV), inp["loc"].to(DEV), inp["attn"].to(DEV),
+                         go.to(DEV))
+    torch.cuda.synchronize()
+    ref = oracle.msda_backward_ref(inp["value"], inp["spatial_shapes"], inp["level_start"],
+                                   inp["loc"], inp["attn"], go)
+    for name, g, r in zip(("grad_value", "grad_loc", "grad_attn"), got, ref):
+        compare(g, r, f"{case} {name}")
