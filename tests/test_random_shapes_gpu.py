@@ -1,6 +1,7 @@
-"""Seeded random small shapes for every forward entry point and the two
-backward calls, each checked element by element against the float64 oracle
-(tests/parity.py tolerances).
+"""Seeded random small shapes for every forward entry point (the DCN and
+MSDA cores, the MSDA reference variants, the fused DCNv4 front end and the
+ContMix core) and the two backward calls. Each is checked element by element
+against the float64 oracle (tests/parity.py tolerances).
 
 The shapes are drawn once from a fixed generator, so the test set is the same
 on every run. They cover the kernels' dispatch decisions between them:
@@ -141,3 +142,46 @@ def test_msda_backward_random_shapes(case):
                                    inp["loc"], inp["attn"], go)
     for name, g, r in zip(("grad_value", "grad_loc", "grad_attn"), got, ref):
         compare(g, r, f"{case} {name}")
+
+
+# ----------------------------------------------- reference variants, front end
+
+@pytest.mark.parametrize("case", _msda_cases(count=6, seed=123), ids=lambda c: "pts_" + "_".join(
+    f"{k}{v}" for k, v in c.items() if k in ("N", "M", "D", "K", "Lq", "dtype")))
+@pytest.mark.parametrize("ref_dim", [2, 4])
+def test_msda_points_random_shapes(case, ref_dim):
+    m = gen.MsdaWorkload("rand", ref_dim=ref_dim, **case)
+    inp = gen.msda_ref_inputs(m, seed=12)
+    d = {k: v.to(DEV) for k, v in inp.items() if torch.is_tensor(v)}
+    out = dcnb.msda_points(d["value"], d["spatial_shapes"], d["level_start"], d["reference"],
+                           d["offsets"], d["attn"], d["valid_ratios"])
+    torch.cuda.synchronize()
+    ref = oracle.msda_points_ref(inp["value"], inp["spatial_shapes"], inp["level_start"],
+                                 inp["reference"], inp["offsets"], inp["attn"],
+                                 inp["valid_ratios"])
+    compare(out, ref, f"{case} ref_dim={ref_dim}")
+
+
+def _fused_cases(count=8, seed=555):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for _ in range(count):
+        G = int(rng.choice([4, 8, 16]))
+        k = int(rng.choice([1, 3]))
+        cases.append(dict(N=int(rng.integers(1, 3)), H=int(rng.integers(2, 20)),
+                          W=int(rng.integers(2, 40)), C=16 * G, G=G, kh=k, kw=k,
+                          pad=(k - 1) // 2, dil=1, dtype=str(rng.choice(["f16", "bf16"]))))
+    return cases
+
+
+@pytest.mark.parametrize("case", _fused_cases(), ids=lambda c: "fused_" + "_".join(
+    f"{k}{v}" for k, v in c.items() if k in ("N", "H", "W", "C", "kh", "dtype")))
+def test_fused_front_end_random_shapes(case):
+    f = gen.FusedWorkload("rand", **case)
+    inp = gen.front_end_inputs(f, seed=13)
+    out = dcnb.dcnv4_fused(inp["x"].to(DEV), inp["w_om"].to(DEV), inp["b_om"].to(DEV),
+                           groups=f.G, kh=f.kh, kw=f.kw, pad=f.pad, dil=f.dil)
+    torch.cuda.synchronize()
+    ref, _, _ = oracle.dcnv4_front_end_ref(inp["x"], inp["w_om"], inp["b_om"], f.kh, f.kw,
+                                           f.pad, f.dil, f.G)
+    compare(out, ref, str(case))
