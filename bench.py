@@ -46,6 +46,10 @@ L1_GATHER_BYTES_PER_CLK = 58.0
 FALLBACK_HBM_GBS = 6650.0
 # Shared memory delivers 32 banks x 4 bytes per SM clock to conflict-free reads.
 SMEM_BYTES_PER_CLK = 128.0
+# Float32 reductions into random 32-byte sectors (two lanes per sector,
+# red.global.add.v4.f32) reach about this many bytes per SM clock on B200
+# (measured with a reduction probe: 120 G sectors/s over 148 SMs at 1965 MHz).
+REDUCTION_BYTES_PER_CLK = 13.2
 
 # DRAM traffic of the timed kernel from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum per launch, headline workload), with the hash of the
@@ -196,6 +200,25 @@ def on_chip_roofline(w, ms_per_launch, sampler, device, band=False):
     return {"bound": "smem" if band else "l1_gather", "achieved": achieved, "peak": peak,
             "unit": "GB/s", "frac": achieved / peak, "gathered_bytes_per_launch": gathered,
             "peak_basis": f"{basis} x {sms} SMs x {mhz} MHz"}
+
+
+def reduction_roofline(w, ms_per_call, sampler, device):
+    """The bound of a DCN backward call: its grad_x scatter adds four corner
+    vectors of D float32 channels per tap, as whole 32-byte sectors at random
+    positions (corners outside the map are skipped, so this slightly
+    overcounts), against the measured random-sector reduction rate x SMs x
+    the median sampled SM clock.  (MSDA's corners are whole 128-byte rows, a
+    pattern this rate does not describe.)"""
+    scattered = w.taps() * 4 * w.D * 4
+    achieved = scattered / (ms_per_call * 1e-3) / 1e9
+    clocks = sampler.summary()
+    mhz = clocks["sm_mhz"] or clocks["sm_max_mhz"] or 1965
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    peak = REDUCTION_BYTES_PER_CLK * sms * mhz * 1e6 / 1e9
+    return {"bound": "l2_reduction", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "reduced_bytes_per_call": scattered,
+            "peak_basis": f"{REDUCTION_BYTES_PER_CLK:g} B/clk/SM measured random-sector float32 "
+                          f"reductions x {sms} SMs x {mhz} MHz"}
 
 
 def fma_roofline(w, ms_per_launch, sampler, device):
@@ -846,7 +869,9 @@ def run_b200(args):
                          "kernel": kernel, "algorithmic_bytes_per_launch": bytes_per_step,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_src == "measured" else "fallback 6.65 TB/s"},
-            "on_chip": (fma_roofline(w, ms_local / args.steps, sampler, device)
+            "on_chip": (reduction_roofline(w, ms_local / args.steps, sampler, device)
+                        if backward and isinstance(w, gen.DcnWorkload)
+                        else fma_roofline(w, ms_local / args.steps, sampler, device)
                         if isinstance(w, gen.DynWorkload)
                         else on_chip_roofline(w, ms_local / args.steps, sampler, device,
                                               band=band)),
