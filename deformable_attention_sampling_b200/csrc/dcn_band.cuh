@@ -56,7 +56,7 @@ namespace dcnb {
 constexpr int kBandMaxStages = 4;
 // Lanes per (pixel, group) item of the band samplers: 1 (each lane reads both
 // 16-byte halves of the group, 16 channels) or 2 (one half each).  Sampler
-// warps per CTA, with the producer warp: 16 warps of up to 128 registers at
+// warps per CTA, with the producer warp: 17 warps of up to 120 registers at
 // one lane per item, 25 warps of up to 72 registers at two.
 #ifndef DCN_BAND_LPI
 #define DCN_BAND_LPI 1
@@ -68,7 +68,7 @@ static_assert(kBandLanesPerItem == 1 || kBandLanesPerItem == 2, "1 or 2 lanes pe
 #define DCN_BAND_AHEAD 1
 #endif
 #ifndef DCN_BAND_WARPS
-#define DCN_BAND_WARPS (DCN_BAND_LPI == 1 ? 15 : 24)
+#define DCN_BAND_WARPS (DCN_BAND_LPI == 1 ? 16 : 24)
 #endif
 constexpr int kBandMaxConsumerWarps = DCN_BAND_WARPS;
 constexpr int kBandMaxThreads = 32 * (kBandMaxConsumerWarps + 1);
