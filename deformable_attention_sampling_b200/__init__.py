@@ -36,6 +36,8 @@ from ._binding import (  # noqa: F401
     dcn_backward_workspace_size,
     dcn_forward,
     dcn_forward_algo,
+    dcn_forward_plan,
+    PLAN_FIELDS,
     DCN_FLAG_BAD_LEVELS,
     DCN_FLAG_OUT_OF_BOUNDS,
     DCN_FLAG_WAIT_TIMEOUT,

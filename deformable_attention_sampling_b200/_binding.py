@@ -26,7 +26,7 @@ DCN_FLAG_WAIT_TIMEOUT = 1
 DCN_FLAG_OUT_OF_BOUNDS = 2
 DCN_FLAG_BAD_LEVELS = 4
 # the entry points the debug library holds (the forward calls and the status calls)
-DEBUG_SYMBOLS = ("dcn_forward", "dcn_forward_algo", "dcnv4_fused_forward",
+DEBUG_SYMBOLS = ("dcn_forward", "dcn_forward_algo", "dcn_forward_plan", "dcnv4_fused_forward",
                  "dcnv4_fused_forward_algo", "msda_forward", "msda_forward_points",
                  "msda_mask_value", "dcn_output_size", "dcn_status_string", "dcn_last_cuda_error",
                  "dcn_launch_count", "dcn_device_flags", "dcn_debug_checks", "dcn_version")
@@ -46,6 +46,7 @@ _LL = ctypes.c_longlong
 SIGNATURES = {
     "dcn_forward": (_I, [_VP, _VP, _VP, _VP] + [_I] * 12 + [_VP]),
     "dcn_forward_algo": (_I, [_VP, _VP, _VP, _VP] + [_I] * 13 + [_VP]),
+    "dcn_forward_plan": (_I, [_I] * 13 + [ctypes.POINTER(ctypes.c_int)]),
     "dcn_device_flags": (_I, [_I]),
     "dcn_debug_checks": (_I, []),
     "msda_forward": (_I, [_VP] * 6 + [_I] * 7 + [_VP]),
@@ -163,6 +164,22 @@ def dcn_forward_algo(x, offset, mask, out, N, H, W, C, G, kh, kw, stride, pad, d
                                     G, kh, kw, stride, pad, dil, softmax_flag, dtype, algo,
                                     _stream(stream)),
            "dcn_forward_algo")
+
+
+PLAN_FIELDS = ("algo", "rows_per_step", "margin", "ring_rows", "sampler_warps",
+               "steps_in_flight", "runs_per_row", "smem_bytes")
+
+
+def dcn_forward_plan(N, H, W, C, G, kh, kw, stride, pad, dil, softmax_flag, dtype,
+                     algo=DCN_ALGO_AUTO, lib=None):
+    """C dcn_forward_plan: the kernel dcn_forward_algo runs for this shape and
+    the band kernel's launch shape, as a dict over PLAN_FIELDS (host only, no
+    GPU needed); raises DcnError on a non-OK status."""
+    plan = (ctypes.c_int * 8)()
+    _check((lib or _load()).dcn_forward_plan(N, H, W, C, G, kh, kw, stride, pad, dil,
+                                             softmax_flag, dtype, algo, plan),
+           "dcn_forward_plan")
+    return dict(zip(PLAN_FIELDS, list(plan)))
 
 
 def dcn_device_flags(reset=False, lib=None):

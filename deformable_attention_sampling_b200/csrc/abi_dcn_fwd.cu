@@ -1,5 +1,6 @@
 // C interface of libdcn_b200.so: dcn_forward and dcn_forward_algo (argument
-// checks, choice between the two forward kernels, launch shape, dispatch).
+// checks, choice between the two forward kernels, launch shape, dispatch), and
+// dcn_forward_plan (the same choice and launch shape, on the host only).
 //
 // Two kernels compute the same operator:
 //   - the band kernel (dcn_band.cuh): input rows staged in shared memory by
@@ -36,16 +37,22 @@ const void* band_kernel_for(int softmax, int kh, int kw) {
                    : (const void*)dcn_band_kernel<T, false, 0>;
 }
 
-// Launch configuration of the band kernel for this call, or false when the
-// shape or the pointers do not qualify.
-bool band_config(const void* x, const void* offset, const void* mask, void* out, int N, int H,
-                 int W, int C, int G, int kh, int kw, int stride, int pad, int dil, int Ho,
-                 int Wo, int es, dcnb::BandArgs* a, int* smem, int* threads) {
+// Launch shape of the band kernel for a problem shape (tensors taken to be
+// 16-byte aligned), or false when the shape does not qualify.  Host only.
+struct BandPlan {
+    int th;              // output rows per step
+    int margin;          // offset margin of the band, rows above and below
+    int ring;            // input rows in the shared-memory ring
+    int warps;           // sampler warps (one more warp produces)
+    int runs_per_row;    // warp runs per output row
+    long long row_bytes, off_row, mask_row, stage, smem;
+};
+
+bool band_plan(int H, int W, int C, int G, int kh, int kw, int stride, int pad, int dil,
+               int Ho, int Wo, int es, BandPlan* p) {
     const int D = C / G;
     const int K = kh * kw;
     if (es != 2 || D != 16 || (C * es) % 128 != 0) return false;
-    if ((((uintptr_t)x | (uintptr_t)offset | (uintptr_t)mask | (uintptr_t)out) % 16) != 0)
-        return false;
     const long long row_bytes = (long long)W * C * es;
     const long long off_row = (long long)Wo * G * K * 2 * es;
     const long long mask_row = (long long)Wo * G * K * es;
@@ -73,46 +80,95 @@ bool band_config(const void* x, const void* offset, const void* mask, void* out,
                                 kBandStepsInFlight * dcnb::kBandDescInts * 4;
         // one step's copies must fit in an mbarrier transaction count
         if (bytes > kBandSmemLimit || band_in_map * row_bytes + stage >= (1 << 20)) continue;
-        a->x = x;
-        a->offset = offset;
-        a->mask = mask;
-        a->out = out;
-        a->H = H;
-        a->W = W;
-        a->C = C;
-        a->G = G;
-        a->kh = kh;
-        a->kw = kw;
-        a->K = K;
-        a->stride = stride;
-        a->pad = pad;
-        a->dil = dil;
-        a->Ho = Ho;
-        a->Wo = Wo;
-        a->rows_total = N * Ho;
-        a->th = th;
-        a->margin = margin;
-        a->ring_rows = (int)ring;
-        a->consumer_warps = warps;
-        a->stages = kBandStepsInFlight;
-        a->runs_per_row = runs_per_row;
-        a->row_bytes = (uint32_t)row_bytes;
-        a->pix_bytes = (uint32_t)(C * es);
-        a->off_row_bytes = (uint32_t)off_row;
-        a->mask_row_bytes = (uint32_t)mask_row;
-        a->ring_bytes = (uint32_t)(ring * row_bytes);
-        a->stage_bytes = (uint32_t)stage;
-        a->div_G = make_div((uint32_t)G);
-        a->div_Ho = make_div((uint32_t)Ho);
-        a->div_runs = make_div((uint32_t)runs_per_row);
-        a->flags = device_flags_word();
-        a->x_bytes = (long long)N * H * row_bytes;
-        a->out_bytes = (long long)N * Ho * Wo * C * es;
-        *smem = (int)bytes;
-        *threads = 32 * (warps + 1);
+        p->th = th;
+        p->margin = margin;
+        p->ring = (int)ring;
+        p->warps = warps;
+        p->runs_per_row = runs_per_row;
+        p->row_bytes = row_bytes;
+        p->off_row = off_row;
+        p->mask_row = mask_row;
+        p->stage = stage;
+        p->smem = bytes;
         return true;
     }
     return false;
+}
+
+// Launch configuration of the band kernel for this call, or false when the
+// shape or the pointers do not qualify.
+bool band_config(const void* x, const void* offset, const void* mask, void* out, int N, int H,
+                 int W, int C, int G, int kh, int kw, int stride, int pad, int dil, int Ho,
+                 int Wo, int es, dcnb::BandArgs* a, int* smem, int* threads) {
+    if ((((uintptr_t)x | (uintptr_t)offset | (uintptr_t)mask | (uintptr_t)out) % 16) != 0)
+        return false;
+    BandPlan p;
+    if (!band_plan(H, W, C, G, kh, kw, stride, pad, dil, Ho, Wo, es, &p)) return false;
+    a->x = x;
+    a->offset = offset;
+    a->mask = mask;
+    a->out = out;
+    a->H = H;
+    a->W = W;
+    a->C = C;
+    a->G = G;
+    a->kh = kh;
+    a->kw = kw;
+    a->K = kh * kw;
+    a->stride = stride;
+    a->pad = pad;
+    a->dil = dil;
+    a->Ho = Ho;
+    a->Wo = Wo;
+    a->rows_total = N * Ho;
+    a->th = p.th;
+    a->margin = p.margin;
+    a->ring_rows = p.ring;
+    a->consumer_warps = p.warps;
+    a->stages = kBandStepsInFlight;
+    a->runs_per_row = p.runs_per_row;
+    a->row_bytes = (uint32_t)p.row_bytes;
+    a->pix_bytes = (uint32_t)(C * es);
+    a->off_row_bytes = (uint32_t)p.off_row;
+    a->mask_row_bytes = (uint32_t)p.mask_row;
+    a->ring_bytes = (uint32_t)(p.ring * p.row_bytes);
+    a->stage_bytes = (uint32_t)p.stage;
+    a->div_G = make_div((uint32_t)G);
+    a->div_Ho = make_div((uint32_t)Ho);
+    a->div_runs = make_div((uint32_t)p.runs_per_row);
+    a->flags = device_flags_word();
+    a->x_bytes = (long long)N * H * p.row_bytes;
+    a->out_bytes = (long long)N * Ho * Wo * C * es;
+    *smem = (int)p.smem;
+    *threads = 32 * (p.warps + 1);
+    return true;
+}
+
+// Argument checks shared by dcn_forward_algo and dcn_forward_plan (shapes,
+// flags, dtype, algo, size limits); the output size on DCN_OK.
+int check_dcn_shape(int N, int H, int W, int C, int G, int kh, int kw, int stride, int pad,
+                    int dil, int softmax_flag, int dtype, int algo, int* Ho_out, int* Wo_out) {
+    const int es = elem_bytes(dtype);
+    if (algo != DCN_ALGO_AUTO && algo != DCN_ALGO_GATHER && algo != DCN_ALGO_BAND)
+        return DCN_ERR_INVALID_ARG;
+    if (es == 0 || N < 0 || H <= 0 || W <= 0 || C <= 0 || G <= 0 || C % G != 0 || kh <= 0 ||
+        kw <= 0 || stride <= 0 || pad < 0 || dil <= 0 || (softmax_flag != 0 && softmax_flag != 1))
+        return DCN_ERR_INVALID_ARG;
+    if (H > kMaxDim || W > kMaxDim || pad > kMaxDim || stride > kMaxDim || dil > kMaxDim ||
+        kh > kMaxDim || kw > kMaxDim || (long long)kh * kw > kMaxTaps)
+        return DCN_ERR_UNSUPPORTED;
+    const int Ho = dcn_output_size(H, kh, stride, pad, dil);
+    const int Wo = dcn_output_size(W, kw, stride, pad, dil);
+    if (Ho <= 0 || Wo <= 0) return DCN_ERR_INVALID_ARG;
+    const long long img_bytes = (long long)H * W * C * es;
+    const long long out_img_bytes = (long long)Ho * Wo * C * es;
+    const long long items = (long long)N * Ho * Wo * G;
+    if (img_bytes > kInt31 || out_img_bytes > kInt31 || items > kInt31 ||
+        (long long)N * Ho * Wo > kInt31)
+        return DCN_ERR_UNSUPPORTED;
+    *Ho_out = Ho;
+    *Wo_out = Wo;
+    return DCN_OK;
 }
 
 template <typename T, int VB>
@@ -147,26 +203,16 @@ extern "C" {
 int dcn_forward_algo(const void* x, const void* offset, const void* mask, void* out, int N,
                      int H, int W, int C, int G, int kh, int kw, int stride, int pad, int dil,
                      int softmax_flag, int dtype, int algo, void* stream) {
+    int Ho = 0, Wo = 0;
+    const int rc = check_dcn_shape(N, H, W, C, G, kh, kw, stride, pad, dil, softmax_flag, dtype,
+                                   algo, &Ho, &Wo);
+    if (rc != DCN_OK) return rc;
     const int es = elem_bytes(dtype);
-    if (algo != DCN_ALGO_AUTO && algo != DCN_ALGO_GATHER && algo != DCN_ALGO_BAND)
-        return DCN_ERR_INVALID_ARG;
-    if (es == 0 || N < 0 || H <= 0 || W <= 0 || C <= 0 || G <= 0 || C % G != 0 || kh <= 0 ||
-        kw <= 0 || stride <= 0 || pad < 0 || dil <= 0 || (softmax_flag != 0 && softmax_flag != 1))
-        return DCN_ERR_INVALID_ARG;
-    if (H > kMaxDim || W > kMaxDim || pad > kMaxDim || stride > kMaxDim || dil > kMaxDim ||
-        kh > kMaxDim || kw > kMaxDim || (long long)kh * kw > kMaxTaps)
-        return DCN_ERR_UNSUPPORTED;
-    const int Ho = dcn_output_size(H, kh, stride, pad, dil);
-    const int Wo = dcn_output_size(W, kw, stride, pad, dil);
-    if (Ho <= 0 || Wo <= 0) return DCN_ERR_INVALID_ARG;
     const int D = C / G;
     const int K = kh * kw;
     const long long img_bytes = (long long)H * W * C * es;
     const long long out_img_bytes = (long long)Ho * Wo * C * es;
     const long long items = (long long)N * Ho * Wo * G;
-    if (img_bytes > kInt31 || out_img_bytes > kInt31 || items > kInt31 ||
-        (long long)N * Ho * Wo > kInt31)
-        return DCN_ERR_UNSUPPORTED;
     if (N == 0) return DCN_OK;
     if (!x || !offset || !mask || !out) return DCN_ERR_INVALID_ARG;
     if ((((uintptr_t)x | (uintptr_t)offset | (uintptr_t)mask | (uintptr_t)out) % es) != 0)
@@ -276,6 +322,38 @@ int dcn_forward_algo(const void* x, const void* offset, const void* mask, void* 
     }
     if (!fn) return DCN_ERR_UNSUPPORTED;
     return launch(fn, a, a.num_tiles, 32 * warps, smem, stream);
+}
+
+int dcn_forward_plan(int N, int H, int W, int C, int G, int kh, int kw, int stride, int pad,
+                     int dil, int softmax_flag, int dtype, int algo, int* plan) {
+    if (!plan) return DCN_ERR_INVALID_ARG;
+    int Ho = 0, Wo = 0;
+    const int rc = check_dcn_shape(N, H, W, C, G, kh, kw, stride, pad, dil, softmax_flag, dtype,
+                                   algo, &Ho, &Wo);
+    if (rc != DCN_OK) return rc;
+    const int es = elem_bytes(dtype);
+    int out[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    BandPlan p;
+    if (algo != DCN_ALGO_GATHER &&
+        band_plan(H, W, C, G, kh, kw, stride, pad, dil, Ho, Wo, es, &p)) {
+        out[0] = DCN_ALGO_BAND;
+        out[1] = p.th;
+        out[2] = p.margin;
+        out[3] = p.ring;
+        out[4] = p.warps;
+        out[5] = kBandStepsInFlight;
+        out[6] = p.runs_per_row;
+        out[7] = (int)p.smem;
+    } else {
+        if (algo == DCN_ALGO_BAND) return DCN_ERR_UNSUPPORTED;
+        const int D = C / G;
+        const int vb = pick_vector_bytes(es, D, 0);
+        if (vb == 0 || D / (vb / es) > 32) return DCN_ERR_UNSUPPORTED;
+        out[0] = DCN_ALGO_GATHER;
+    }
+    if (N == 0) out[0] = DCN_ALGO_AUTO;   // nothing is launched
+    for (int i = 0; i < 8; ++i) plan[i] = out[i];
+    return DCN_OK;
 }
 
 int dcn_forward(const void* x, const void* offset, const void* mask, void* out, int N, int H,

@@ -124,6 +124,33 @@ DCN_API int dcn_forward_algo(const void* x, const void* offset, const void* mask
                      int algo, void* stream);
 
 /*
+ * dcn_forward_plan - which kernel dcn_forward_algo runs for a shape, and the
+ * band kernel's launch shape.  Host only: no CUDA call, no device memory.
+ *
+ * Arguments as dcn_forward_algo without the tensors and the stream; the
+ * tensors are taken to be 16-byte aligned.  `plan` (caller-owned, 8 ints) is
+ * written on DCN_OK only:
+ *   plan[0]  DCN_ALGO_BAND or DCN_ALGO_GATHER, the kernel that runs; 0 when
+ *            N = 0 (nothing is launched; plan[1..7] still describe the shape)
+ *   plan[1]  band kernel: output rows per step            (0 for the gather kernel)
+ *   plan[2]  band kernel: offset margin, input rows staged above and below
+ *            the window rows
+ *   plan[3]  band kernel: input rows in the shared-memory ring
+ *   plan[4]  band kernel: sampler warps per CTA (one more warp issues the copies)
+ *   plan[5]  band kernel: steps in flight
+ *   plan[6]  band kernel: warp runs (32 items) per output row
+ *   plan[7]  band kernel: dynamic shared memory per CTA, bytes
+ * A CTA of the band kernel owns a contiguous range of output rows (numbered
+ * n * Ho + oy over the batch), one CTA per SM.
+ * Errors: those of dcn_forward_algo that the shape decides (DCN_ERR_INVALID_ARG,
+ * DCN_ERR_UNSUPPORTED, including DCN_ALGO_BAND on a shape the band kernel
+ * does not take), and DCN_ERR_INVALID_ARG for a null `plan`.
+ */
+DCN_API int dcn_forward_plan(int N, int H, int W, int C, int G, int kh, int kw,
+                     int stride, int pad, int dil, int softmax_flag, int dtype,
+                     int algo, int* plan);
+
+/*
  * dcn_device_flags - the per-device status word of the library's kernels.
  *
  * Bits (sticky until reset):
