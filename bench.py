@@ -50,6 +50,11 @@ SMEM_BYTES_PER_CLK = 128.0
 # red.global.add.v4.f32) reach about this many bytes per SM clock on B200
 # (measured with a reduction probe: 120 G sectors/s over 148 SMs at 1965 MHz).
 REDUCTION_BYTES_PER_CLK = 13.2
+# Random 128-byte rows (four lanes of 32 bytes each, ld.global.nc) gathered
+# from a 40 MB L2-resident float32 tensor reach about this many bytes per SM
+# clock on B200 (measured: 141 G rows/s over 148 SMs at 1965 MHz; TMA
+# tile::gather4 loads of the same rows reached at most 46 G rows/s).
+ROW_GATHER_BYTES_PER_CLK = 62.0
 
 # DRAM traffic of the timed kernel from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum per launch, headline workload), with the hash of the
@@ -219,6 +224,25 @@ def reduction_roofline(w, ms_per_call, sampler, device):
             "frac": achieved / peak, "reduced_bytes_per_call": scattered,
             "peak_basis": f"{REDUCTION_BYTES_PER_CLK:g} B/clk/SM measured random-sector float32 "
                           f"reductions x {sms} SMs x {mhz} MHz"}
+
+
+def row_gather_roofline(w, ms_per_launch, sampler, device):
+    """The SM-side bound of an MSDA forward: every tap reads four corner rows
+    of D channels (a (pixel, head) row of the value tensor, out-of-map ones
+    from a clamped row with zero weight), at data-dependent positions in a
+    value tensor that stays in L2, against the measured rate of random
+    128-byte row gathers from L2 x SMs x the median sampled SM clock."""
+    es = gen.DTYPES[w.dtype].itemsize
+    gathered = w.taps() * 4 * w.D * es
+    achieved = gathered / (ms_per_launch * 1e-3) / 1e9
+    clocks = sampler.summary()
+    mhz = clocks["sm_mhz"] or clocks["sm_max_mhz"] or 1965
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    peak = ROW_GATHER_BYTES_PER_CLK * sms * mhz * 1e6 / 1e9
+    return {"bound": "l2_row_gather", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "gathered_bytes_per_launch": gathered,
+            "peak_basis": f"{ROW_GATHER_BYTES_PER_CLK:g} B/clk/SM measured random 128-byte row "
+                          f"gathers from L2 x {sms} SMs x {mhz} MHz"}
 
 
 def fma_roofline(w, ms_per_launch, sampler, device):
@@ -873,6 +897,8 @@ def run_b200(args):
                         if backward and isinstance(w, gen.DcnWorkload)
                         else fma_roofline(w, ms_local / args.steps, sampler, device)
                         if isinstance(w, gen.DynWorkload)
+                        else row_gather_roofline(w, ms_local / args.steps, sampler, device)
+                        if isinstance(w, gen.MsdaWorkload) and not backward
                         else on_chip_roofline(w, ms_local / args.steps, sampler, device,
                                               band=band)),
             "e2e": {"value": taps_total / (e2e_ms * 1e-3), "unit": "taps/s",
