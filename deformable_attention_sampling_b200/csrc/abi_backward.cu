@@ -413,7 +413,7 @@ namespace {
 constexpr long long kStaticScratchBytes = DCN_STATIC_SCRATCH_BYTES;   // 16 MiB
 constexpr int kMaxScratchDevices = 64;
 
-__device__ __align__(256) float g_static_scratch[kStaticScratchBytes / 4];
+static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / 4];
 
 std::mutex g_scratch_mutex;
 void* g_scratch_ptr[kMaxScratchDevices] = {};

@@ -26,11 +26,13 @@
 // Work decomposition (one CTA = 8 output rows x 32 columns of one group and
 // one 16-channel chunk; 8 warps):
 //   warp  = one output row, as two blocks of 16 columns;
-//   lane  = one location (column) of the row for the softmax: it copies its
-//           own numbers of kernel row ky + 1 into its own slot (8-byte
-//           cp.async, no barrier) while it reads row ky, updates its running
-//           maximum and sum (online softmax, as the SIMT kernel), and writes
-//           its band of A (high and low parts) for both k-steps;
+//   lane  = one location (column) of the row for the softmax: the numbers of
+//           kernel row ky + 1 of the warp's 32 locations are copied into
+//           their slots (8-byte cp.async; at K = 13 four lanes per location,
+//           at K = 7 each lane its own; warp barriers only) while each lane
+//           reads its location's row ky, updates its running maximum and sum
+//           (online softmax, as the SIMT kernel), and writes its band of A
+//           (high and low parts) for both k-steps;
 //   mma   = per block and k-step: A (ldmatrix.x4, high and low), B
 //           (ldmatrix.x4.trans: 16 window columns x 16 channels), four
 //           m16n8k16 products into float32 accumulators (16 per lane).
@@ -227,23 +229,58 @@ __global__ void __launch_bounds__(kMmaThreads, 2) dynconv_mma_kernel(const DynAr
     const int w_col = a.G * K * K;
     const int w_row = a.W * w_col;
     auto in_map = [&](int row, int col) { return y0 + row < a.H && x0 + col < a.W; };
-    // Each thread copies and reads the numbers of its own location (warp, lane)
-    // only, so the raw buffers need no barrier: kernel row ky goes to buffer
-    // ky & 1 as 8-byte units from the one holding the row's first number, the
-    // last clipped to the row's end.
+    // A warp stages the numbers of its own row's 32 locations; each thread then
+    // reads those of its own location (warp, lane).  Kernel row ky goes to
+    // buffer ky & 1 as 8-byte units from the one holding the row's first
+    // number, the last clipped to the row's end.  The 32 locations' rows sit
+    // w_col numbers apart in global memory, so a copy instruction whose lanes
+    // take one location each touches 32 lines.
     const bool mine = in_map(warp, lane);
-    const char* my_w = reinterpret_cast<const char*>(wt + warp * w_row + lane * w_col);
-    const uint32_t my_slot = (uint32_t)__cvta_generic_to_shared(raw) +
-                             (uint32_t)((warp * kMmaCols + lane) * SW * 4);
+    const char* row_w = reinterpret_cast<const char*>(wt + warp * w_row);
+    const char* my_w = row_w + (long long)lane * w_col * es;
+    const uint32_t row_slot = (uint32_t)__cvta_generic_to_shared(raw) +
+                              (uint32_t)(warp * kMmaCols * SW * 4);
+    const uint32_t my_slot = row_slot + (uint32_t)(lane * SW * 4);
+    // units a kernel row can span (from the 8-byte unit of its first number)
+    constexpr int NUC = (2 * K + 6 + 7) / 8;
+    // Four units (K = 13): four lanes per location, one unit each, so a copy
+    // instruction touches eight locations' lines (247.8 -> 238.4 us per
+    // 64 x 56 x 56 x 64 launch).  Three units (K = 7): a lane per location
+    // (the packed mapping of 32 x 3 units measured 127.0 against 123.0 us).
+    constexpr bool kWarpCopy = NUC >= 4;
     auto copy_row = [&](int ky) {
-        if (mine) {
-            const char* first = my_w + ky * K * es;
-            const char* last = first + K * es;
-            const char* u8 = reinterpret_cast<const char*>((uintptr_t)first & ~(uintptr_t)7);
-            uint32_t dst = my_slot + (uint32_t)((ky & 1) * NP * SW * 4);
-            for (; u8 < last; u8 += 8, dst += 8) {
-                const long long left = last - u8;
-                cp_async8(dst, u8, left >= 8 ? 8u : (uint32_t)left);
+        if constexpr (!kWarpCopy) {
+            // each thread its own location's units
+            if (mine) {
+                const char* first = my_w + ky * K * es;
+                const char* last = first + K * es;
+                const char* u8 = reinterpret_cast<const char*>((uintptr_t)first & ~(uintptr_t)7);
+                uint32_t dst = my_slot + (uint32_t)((ky & 1) * NP * SW * 4);
+                for (; u8 < last; u8 += 8, dst += 8) {
+                    const long long left = last - u8;
+                    cp_async8(dst, u8, left >= 8 ? 8u : (uint32_t)left);
+                }
+            }
+        } else {
+            // UPL lanes per location: copy f of the row's 32 x UPL (location,
+            // unit) pairs is location f / UPL, unit f % UPL
+            constexpr int UPL = NUC <= 4 ? 4 : 8;
+#pragma unroll
+            for (int pass = 0; pass < UPL; ++pass) {
+                const int f = pass * 32 + lane;
+                const int col = f / UPL, unit = f - col * UPL;
+                if (in_map(warp, col)) {
+                    const char* first = row_w + ((long long)col * w_col + ky * K) * es;
+                    const char* last = first + K * es;
+                    const char* u8 = reinterpret_cast<const char*>((uintptr_t)first &
+                                                                   ~(uintptr_t)7) + 8 * unit;
+                    if (u8 < last) {
+                        const long long left = last - u8;
+                        const uint32_t dst = row_slot + (uint32_t)(col * SW * 4) +
+                                             (uint32_t)((ky & 1) * NP * SW * 4) + 8u * unit;
+                        cp_async8(dst, u8, left >= 8 ? 8u : (uint32_t)left);
+                    }
+                }
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
@@ -290,14 +327,17 @@ __global__ void __launch_bounds__(kMmaThreads, 2) dynconv_mma_kernel(const DynAr
     __syncthreads();   // the window (every warp's copies) and the zeroed A tiles
 #pragma unroll 1
     for (int ky = 0; ky < K; ++ky) {
-        // this thread's row ky + 1 in flight while row ky is used; buffer
-        // (ky + 1) & 1 was last read by this same thread, at row ky - 1
+        // the warp's row ky + 1 in flight while row ky is used; buffer
+        // (ky + 1) & 1 was last read at row ky - 1, by every lane of the warp
+        // before this barrier
+        __syncwarp();
         if (ky + 1 < K) {
             copy_row(ky + 1);
             asm volatile("cp.async.wait_group 1;" ::: "memory");
         } else {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
+        __syncwarp();   // every lane's copies of row ky have landed
 
         // this location's numbers of kernel row ky (0 outside the map)
         float e[2 * NWORD];
