@@ -43,7 +43,7 @@ bool band_fused_config(const void* x, const void* w_om, const void* b_om, void* 
     const int row_items = W * G;
     const int run_items = 32 / dcnb::kBandLanesPerItem;
     const int runs_per_row = (row_items + run_items - 1) / run_items;
-    const int consumer_warps = 16 - 2 - dcnb::kFusedEpilogueWarps;
+    const int consumer_warps = dcnb::kFusedMaxThreads / 32 - 2 - dcnb::kFusedEpilogueWarps;
     const uint32_t w_bytes = (uint32_t)kchunks * (uint32_t)NJ * 128u;
     const uint32_t om_stride = (uint32_t)((J + 3) / 4 * 4);
     // candidates in order of preference: offset margin (taps that leave the
