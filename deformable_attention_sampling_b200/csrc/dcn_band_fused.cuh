@@ -36,12 +36,12 @@
 namespace dcnb {
 
 constexpr int kFusedEpilogueWarps = 4;
-// Warps per CTA: 14 samplers, the producer, the MMA warp and 4 epilogue warps
-// (measured on the 64 x 56 x 56 x 64 fp16 front end: 133.8 us per launch
-// with 14 samplers, 137.6 with 10, 137.7 with 12, 147.2 with 16 and 142.3
-// with 18, the last two spilling at their register limit).
+// Warps per CTA: 10 samplers, the producer, the MMA warp and 4 epilogue
+// warps.  Measured on the 64 x 56 x 56 x 64 fp16 front end with the tap loop
+// not unrolled, us per launch: 114.0 with 10 samplers, 117.6 with 14, 128.2
+// with 18 (with the taps unrolled: 137.6 / 133.8 / 142.3).
 #ifndef DCN_FUSED_WARPS
-#define DCN_FUSED_WARPS 20
+#define DCN_FUSED_WARPS 16
 #endif
 constexpr int kFusedMaxThreads = 32 * DCN_FUSED_WARPS;
 
