@@ -38,8 +38,9 @@ namespace dcnb {
 constexpr int kFusedEpilogueWarps = 4;
 // Warps per CTA: 10 samplers, the producer, the MMA warp and 4 epilogue
 // warps.  Measured on the 64 x 56 x 56 x 64 fp16 front end with the tap loop
-// not unrolled, us per launch: 114.0 with 10 samplers, 117.6 with 14, 128.2
-// with 18 (with the taps unrolled: 137.6 / 133.8 / 142.3).
+// not unrolled, us per launch: 114.0 with 10 samplers, 120.8 with 12, 117.6
+// with 14, 128.2 with 18 (with the taps unrolled: 137.6 / 137.7 / 133.8 /
+// 142.3).
 #ifndef DCN_FUSED_WARPS
 #define DCN_FUSED_WARPS 16
 #endif
